@@ -1,0 +1,425 @@
+// libi8q: the C ABI declared in include/i8q.h.  Host-side argument checks, launch
+// configuration, TMA tensor-map encoding; all arithmetic of the method runs in the kernels
+// included below.  Built as a single translation unit so that the device error word is one
+// symbol per device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <climits>
+#include <mutex>
+
+#include "../../include/i8q.h"
+#include "common.cuh"
+#include "gemm_w8a16.cuh"
+#include "gemm_w8a8.cuh"
+#include "quant.cuh"
+
+namespace i8q {
+
+// ------------------------------------------------------------------ error text --------------
+static thread_local char t_last_error[256] = "";
+
+static i8q_status cuda_fail(cudaError_t e, const char* what) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%d)", what, cudaGetErrorString(e), (int)e);
+  return I8Q_ERR_CUDA;
+}
+
+#define I8Q_CUDA(call)                                   \
+  do {                                                   \
+    cudaError_t e_ = (call);                             \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call);  \
+  } while (0)
+
+#define I8Q_LAUNCHED(what)                                    \
+  do {                                                        \
+    cudaError_t e_ = cudaGetLastError();                      \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what);        \
+  } while (0)
+
+// ------------------------------------------------------------------ device info -------------
+struct DeviceInfo {
+  int ok = -1;   // -1 unknown, 0 unsupported, 1 supported
+  int sms = 0;
+};
+static constexpr int kMaxDevices = 64;
+static DeviceInfo g_dev[kMaxDevices];
+static std::mutex g_dev_mu;
+
+static i8q_status current_device(int* sms) {
+  int dev = 0;
+  I8Q_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return I8Q_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.ok < 0) {
+    int major = 0, minor = 0, n = 0;
+    I8Q_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    I8Q_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    I8Q_CUDA(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev));
+    d.ok = (major == 10 && minor == 0) ? 1 : 0;
+    d.sms = n;
+    if (!d.ok)
+      snprintf(t_last_error, sizeof(t_last_error), "device %d is sm_%d%d; libi8q is built for sm_100a", dev, major,
+               minor);
+  }
+  if (!d.ok) return I8Q_ERR_UNSUPPORTED;
+  *sms = d.sms;
+  return I8Q_OK;
+}
+
+// ------------------------------------------------------------------ TMA tensor maps ---------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows][cols] of `elem` bytes, box = box_rows x box_cols, given swizzle.
+static i8q_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem,
+                               uint64_t rows, uint64_t cols, uint64_t ld_elems, uint32_t box_rows,
+                               uint32_t box_cols, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled is unavailable");
+    return I8Q_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld_elems * (uint64_t)elem};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return I8Q_ERR_CUDA;
+  }
+  return I8Q_OK;
+}
+
+// ------------------------------------------------------------------ argument checks ---------
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define I8Q_REQUIRE(cond, code)  \
+  do {                           \
+    if (!(cond)) return (code);  \
+  } while (0)
+
+static inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+template <typename Kern>
+static i8q_status set_smem(Kern k, int bytes) {
+  I8Q_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  return I8Q_OK;
+}
+
+static constexpr int64_t kMaxDim = (int64_t)1 << 30;
+
+// ------------------------------------------------------------------ W8A16 launch ------------
+// Split-K factor: the cluster size s in 1..8 minimising (waves of CTAs) x (slabs per CTA).
+static int w8a16_splits(int64_t tiles, int64_t KB, int sms) {
+  int best = 1;
+  int64_t best_cost = INT64_MAX;
+  for (int s = 1; s <= 8 && s <= KB; ++s) {
+    const int64_t cost = cdiv(tiles * s, sms) * cdiv(KB, s);
+    if (cost < best_cost) { best_cost = cost; best = s; }
+  }
+  return best;
+}
+
+template <int MP>
+static i8q_status launch_w8a16_mp(const uint16_t* x, const int8_t* wq, const uint16_t* s, int M, int N, int K,
+                                  uint16_t* y, int sms, cudaStream_t stream) {
+  using C = W8A16Cfg<MP>;
+  auto kern = k_gemm_w8a16<MP>;
+  static std::once_flag once;
+  static i8q_status attr = I8Q_OK;
+  std::call_once(once, [&] { attr = set_smem(kern, C::SMEM_BYTES); });
+  if (attr) return attr;
+  CUtensorMap tw, tx;
+  i8q_status st = make_tmap_2d(&tw, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, W8A16_BN, 128,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  st = make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, K, K, MP, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  const int64_t tiles = cdiv(N, W8A16_BN);
+  const int splits = w8a16_splits(tiles, K / 128, sms);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits, 1);
+  cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = (unsigned)splits;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  W8A16Args a{s, M, N, K, y};
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, tw, tx, a));
+  return I8Q_OK;
+}
+
+static i8q_status launch_w8a16(const uint16_t* x, const int8_t* wq, const uint16_t* s, int M, int N, int K,
+                               uint16_t* y, int sms, cudaStream_t stream) {
+  if (M <= 16) return launch_w8a16_mp<16>(x, wq, s, M, N, K, y, sms, stream);
+  if (M <= 32) return launch_w8a16_mp<32>(x, wq, s, M, N, K, y, sms, stream);
+  return launch_w8a16_mp<64>(x, wq, s, M, N, K, y, sms, stream);
+}
+
+// ------------------------------------------------------------------ W8A8 launch -------------
+static i8q_status gemm_w8a8_common_checks(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                                          int64_t M, int64_t N, int64_t K, const void* y, const void* dbg) {
+  I8Q_REQUIRE(M >= 0 && N >= 0 && K >= 0 && M < kMaxDim && N < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(K % 128 == 0 && N % 8 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(127LL * 127LL * K < (1LL << 31), I8Q_ERR_SHAPE);
+  if (M == 0 || N == 0) return I8Q_OK;
+  I8Q_REQUIRE(y, I8Q_ERR_NULL);
+  I8Q_REQUIRE(aligned16(y) && aligned16(dbg), I8Q_ERR_ALIGN);
+  if (K == 0) return I8Q_OK;
+  I8Q_REQUIRE(xq && sx && wq && sw, I8Q_ERR_NULL);
+  I8Q_REQUIRE(aligned16(xq) && aligned16(sx) && aligned16(wq) && aligned16(sw), I8Q_ERR_ALIGN);
+  return I8Q_OK;
+}
+
+template <int BN, bool BLOCKWISE, bool F32, bool DBG>
+static i8q_status launch_w8a8(const CUtensorMap& ta, const CUtensorMap& tb, const W8A8Args& a, int sms,
+                              cudaStream_t s) {
+  using C = W8A8Cfg<BN>;
+  auto kern = k_gemm_w8a8<BN, BLOCKWISE, F32, DBG>;
+  static std::once_flag once;
+  static i8q_status attr = I8Q_OK;
+  std::call_once(once, [&] { attr = set_smem(kern, C::SMEM_BYTES); });
+  if (attr) return attr;
+  const int64_t tiles = cdiv(a.M, GEMM_BM) * cdiv(a.N, BN);
+  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+  kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, s>>>(ta, tb, a);
+  I8Q_LAUNCHED("k_gemm_w8a8");
+  return I8Q_OK;
+}
+
+}  // namespace i8q
+
+using namespace i8q;
+
+// ================================================================== entry points =============
+extern "C" {
+
+int i8q_version(void) { return 100; }
+
+const char* i8q_status_string(i8q_status s) {
+  switch (s) {
+    case I8Q_OK: return "I8Q_OK";
+    case I8Q_ERR_NULL: return "I8Q_ERR_NULL";
+    case I8Q_ERR_SHAPE: return "I8Q_ERR_SHAPE";
+    case I8Q_ERR_ALIGN: return "I8Q_ERR_ALIGN";
+    case I8Q_ERR_DTYPE: return "I8Q_ERR_DTYPE";
+    case I8Q_ERR_CUDA: return "I8Q_ERR_CUDA";
+    case I8Q_ERR_TIMEOUT: return "I8Q_ERR_TIMEOUT";
+    case I8Q_ERR_UNSUPPORTED: return "I8Q_ERR_UNSUPPORTED";
+  }
+  return "I8Q_ERR_UNKNOWN";
+}
+
+const char* i8q_last_error_string(void) { return t_last_error; }
+
+i8q_status i8q_status_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(S(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int word = 0, zero = 0;
+  I8Q_CUDA(cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)));
+  if (word != 0) {
+    I8Q_CUDA(cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)));
+    snprintf(t_last_error, sizeof(t_last_error), "bounded device wait expired (site %u)", (word >> 8) & 0xFFu);
+    return I8Q_ERR_TIMEOUT;
+  }
+  return I8Q_OK;
+}
+
+// ---------------------------------------------------------------- a1 -------------------------
+i8q_status i8q_quant_act_token_group(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int8_t* xq, float* sx,
+                                     int64_t ld_sx, void* stream) {
+  I8Q_REQUIRE(M >= 0 && K >= 0 && M < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(K % 128 == 0, I8Q_ERR_SHAPE);
+  if (M == 0 || K == 0) return I8Q_OK;
+  I8Q_REQUIRE(x && xq && sx, I8Q_ERR_NULL);
+  I8Q_REQUIRE(ldx >= K && ldx % 8 == 0 && ld_sx >= M && ld_sx % 4 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(aligned16(x) && aligned16(xq) && aligned16(sx), I8Q_ERR_ALIGN);
+  int sms;
+  i8q_status st = current_device(&sms);
+  if (st) return st;
+  const int64_t KB = K / 128;
+  const int64_t pairs = (M * KB + 1) / 2;
+  const int64_t warps_needed = (pairs + 1) / 2;                 // two pairs in flight per warp
+  int64_t blocks = (warps_needed + 7) / 8;
+  const int64_t cap = (int64_t)sms * 8;                          // 8 CTAs x 256 threads per SM
+  if (blocks > cap) blocks = cap;
+  k_quant_act_token_group<<<(unsigned)blocks, 256, 0, S(stream)>>>(x, M, KB, ldx, xq, sx, ld_sx);
+  I8Q_LAUNCHED("k_quant_act_token_group");
+  return I8Q_OK;
+}
+
+// ---------------------------------------------------------------- a2 -------------------------
+i8q_status i8q_quant_act_token(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int8_t* xq, float* sx,
+                               void* stream) {
+  I8Q_REQUIRE(M >= 0 && K >= 0 && M < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(K % 16 == 0, I8Q_ERR_SHAPE);
+  if (M == 0) return I8Q_OK;
+  I8Q_REQUIRE(x && xq && sx, I8Q_ERR_NULL);
+  I8Q_REQUIRE(ldx >= K && ldx % 8 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(aligned16(x) && aligned16(xq) && aligned16(sx), I8Q_ERR_ALIGN);
+  int sms;
+  i8q_status st = current_device(&sms);
+  if (st) return st;
+  const int64_t nv = K / 8;
+  const unsigned grid = (unsigned)M;
+  if (nv <= 128 * 1)
+    k_quant_act_token<1><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
+  else if (nv <= 128 * 2)
+    k_quant_act_token<2><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
+  else if (nv <= 128 * 4)
+    k_quant_act_token<4><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
+  else if (nv <= 128 * 8)
+    k_quant_act_token<8><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
+  else if (nv <= 128 * 16)
+    k_quant_act_token<16><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
+  else
+    k_quant_act_token<0><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
+  I8Q_LAUNCHED("k_quant_act_token");
+  return I8Q_OK;
+}
+
+// ---------------------------------------------------------------- a3', a3 --------------------
+i8q_status i8q_quant_weight_block(const uint16_t* w, int64_t N, int64_t K, int8_t* wq, float* sw, void* stream) {
+  I8Q_REQUIRE(N >= 0 && K >= 0 && N < kMaxDim && K < kMaxDim && K % 128 == 0, I8Q_ERR_SHAPE);
+  if (N == 0 || K == 0) return I8Q_OK;
+  I8Q_REQUIRE(w && wq && sw, I8Q_ERR_NULL);
+  I8Q_REQUIRE(aligned16(w) && aligned16(wq) && aligned16(sw), I8Q_ERR_ALIGN);
+  int sms;
+  i8q_status st = current_device(&sms);
+  if (st) return st;
+  const int64_t blocks = cdiv(N, 128) * (K / 128);
+  k_quant_weight_block<false><<<(unsigned)blocks, 256, 0, S(stream)>>>(w, nullptr, N, K, wq, sw);
+  I8Q_LAUNCHED("k_quant_weight_block<bf16>");
+  return I8Q_OK;
+}
+
+i8q_status i8q_requant_fp8_to_int8_block(const uint8_t* w, const float* sf, int64_t N, int64_t K, int8_t* wq,
+                                         float* sw, void* stream) {
+  I8Q_REQUIRE(N >= 0 && K >= 0 && N < kMaxDim && K < kMaxDim && K % 128 == 0, I8Q_ERR_SHAPE);
+  if (N == 0 || K == 0) return I8Q_OK;
+  I8Q_REQUIRE(w && sf && wq && sw, I8Q_ERR_NULL);
+  I8Q_REQUIRE(aligned16(w) && aligned16(sf) && aligned16(wq) && aligned16(sw), I8Q_ERR_ALIGN);
+  int sms;
+  i8q_status st = current_device(&sms);
+  if (st) return st;
+  const int64_t blocks = cdiv(N, 128) * (K / 128);
+  k_quant_weight_block<true><<<(unsigned)blocks, 256, 0, S(stream)>>>(w, sf, N, K, wq, sw);
+  I8Q_LAUNCHED("k_quant_weight_block<e4m3>");
+  return I8Q_OK;
+}
+
+i8q_status i8q_requant_fp8_to_int8_channel(const uint8_t* w, const float* sf, int64_t N, int64_t K, int8_t* wq,
+                                           float* sw, void* stream) {
+  I8Q_REQUIRE(N >= 0 && K >= 0 && N < kMaxDim && K < kMaxDim && K % 128 == 0, I8Q_ERR_SHAPE);
+  if (N == 0) return I8Q_OK;
+  I8Q_REQUIRE(w && sf && wq && sw, I8Q_ERR_NULL);
+  I8Q_REQUIRE(aligned16(w) && aligned16(sf) && aligned16(wq) && aligned16(sw), I8Q_ERR_ALIGN);
+  int sms;
+  i8q_status st = current_device(&sms);
+  if (st) return st;
+  k_requant_fp8_channel<<<(unsigned)N, 128, 0, S(stream)>>>(w, sf, K, wq, sw);
+  I8Q_LAUNCHED("k_requant_fp8_channel");
+  return I8Q_OK;
+}
+
+// ---------------------------------------------------------------- a4, a5 ---------------------
+i8q_status i8q_gemm_w8a8_channel(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw, int64_t M,
+                                 int64_t N, int64_t K, uint16_t* y, int32_t* dbg, void* stream) {
+  i8q_status st = gemm_w8a8_common_checks(xq, sx, wq, sw, M, N, K, y, dbg);
+  if (st || M == 0 || N == 0) return st;
+  int sms;
+  st = current_device(&sms);
+  if (st) return st;
+  if (K == 0) {
+    I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * 2, S(stream)));
+    if (dbg) I8Q_CUDA(cudaMemsetAsync(dbg, 0, (size_t)M * N * 4, S(stream)));
+    return I8Q_OK;
+  }
+  constexpr int BN = 256;
+  CUtensorMap ta, tb;
+  st = make_tmap_2d(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, GEMM_BM, GEMM_BK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  st = make_tmap_2d(&tb, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, BN, GEMM_BK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  W8A8Args a{sx, 0, sw, (int)M, (int)N, (int)K, y, dbg};
+  if (dbg) return launch_w8a8<BN, false, false, true>(ta, tb, a, sms, S(stream));
+  return launch_w8a8<BN, false, false, false>(ta, tb, a, sms, S(stream));
+}
+
+i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx, const int8_t* wq, const float* sw,
+                               int64_t M, int64_t N, int64_t K, void* y, i8q_out_dtype out, int32_t* dbg,
+                               void* stream) {
+  I8Q_REQUIRE(out == I8Q_OUT_BF16 || out == I8Q_OUT_FP32, I8Q_ERR_DTYPE);
+  i8q_status st = gemm_w8a8_common_checks(xq, sx, wq, sw, M, N, K, y, dbg);
+  if (st || M == 0 || N == 0) return st;
+  if (K > 0) I8Q_REQUIRE(ld_sx >= M && ld_sx % 4 == 0, I8Q_ERR_SHAPE);
+  int sms;
+  st = current_device(&sms);
+  if (st) return st;
+  const size_t osz = out == I8Q_OUT_FP32 ? 4 : 2;
+  if (K == 0) {
+    I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * osz, S(stream)));
+    return I8Q_OK;
+  }
+  constexpr int BN = 128;
+  CUtensorMap ta, tb;
+  st = make_tmap_2d(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, GEMM_BM, GEMM_BK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  st = make_tmap_2d(&tb, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, BN, GEMM_BK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  W8A8Args a{sx, ld_sx, sw, (int)M, (int)N, (int)K, y, dbg};
+  const bool f32 = out == I8Q_OUT_FP32;
+  if (dbg) {
+    if (f32) return launch_w8a8<BN, true, true, true>(ta, tb, a, sms, S(stream));
+    return launch_w8a8<BN, true, false, true>(ta, tb, a, sms, S(stream));
+  }
+  if (f32) return launch_w8a8<BN, true, true, false>(ta, tb, a, sms, S(stream));
+  return launch_w8a8<BN, true, false, false>(ta, tb, a, sms, S(stream));
+}
+
+// ---------------------------------------------------------------- a6 -------------------------
+i8q_status i8q_gemm_w8a16_group(const uint16_t* x, const int8_t* wq, const uint16_t* s, int64_t M, int64_t N,
+                                int64_t K, uint16_t* y, void* stream) {
+  I8Q_REQUIRE(M >= 0 && N >= 0 && K >= 0 && N < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(M <= W8A16_MAX_M && K % 128 == 0 && N % 8 == 0, I8Q_ERR_SHAPE);
+  if (M == 0 || N == 0) return I8Q_OK;
+  I8Q_REQUIRE(y, I8Q_ERR_NULL);
+  I8Q_REQUIRE(aligned16(y), I8Q_ERR_ALIGN);
+  int sms;
+  i8q_status st = current_device(&sms);
+  if (st) return st;
+  if (K == 0) {
+    I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * 2, S(stream)));
+    return I8Q_OK;
+  }
+  I8Q_REQUIRE(x && wq && s, I8Q_ERR_NULL);
+  I8Q_REQUIRE(aligned16(x) && aligned16(wq) && aligned16(s), I8Q_ERR_ALIGN);
+  return launch_w8a16(x, wq, s, (int)M, (int)N, (int)K, y, sms, S(stream));
+}
+
+}  // extern "C"
