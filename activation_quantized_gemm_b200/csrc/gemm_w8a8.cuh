@@ -5,18 +5,28 @@
 //    the per-token x per-output-channel scale once and writes bf16.
 //  * block-wise (Fig. 3 left): every 128-wide K slab gets a fresh TMEM accumulator; the epilogue
 //    warps read each slab's exact int32 partial sum and fold it into an fp32 running sum with the
-//    slab's activation-group x weight-block scale ("several dequantizations inside the INT8
+//    slab's activation-group x weight-block scale (the "several dequantizations inside the INT8
 //    matmul, on the CUDA cores").  Two TMEM accumulator buffers let the tensor core run the next
 //    slab while the CUDA cores dequantize the previous one.
 //
-// Kernel structure (persistent, one CTA per SM, 256 threads):
-//   warp 0      : TMA producer - 128x128 activation tile + BNx128 weight tile per slab into a
-//                 STAGES-deep ring of 128B-swizzled shared-memory buffers (mbarrier complete_tx).
-//   warp 1      : TMEM allocator and MMA issuer - 4 x tcgen05.mma (K = 32 each) per slab,
-//                 tcgen05.commit frees the smem stage and hands the accumulator to the epilogue.
-//   warps 4..7  : epilogue - warp w reads TMEM lanes 32*(w%4).. (tile rows), one row per thread.
-// Tiles are 128 tokens x BN output channels, visited in bands of 16 token-blocks so that the
-// activations and weights the 148 CTAs touch at one time stay resident in L2.
+// Kernel structure: persistent, one CTA pair (thread-block cluster of 2) per 2 SMs, each pair
+// computes 256 x BN output tiles with the pair-wide MMA (tcgen05 cta_group::2, M = 256):
+// CTA r of the pair stages token rows [128 r, 128 r + 128) of the tile's activations and weight
+// rows [BN/2 r, BN/2 (r + 1)) of its weights, so each SM streams 128 + BN/2 rows per K slab for
+// 128 x BN outputs.  12 warps per CTA:
+//   warp 0       TMA producer (both CTAs): per slab, own activation + weight halves into a
+//                STAGES-deep ring of 128B-swizzled buffers; completion is counted on the leader
+//                CTA's barrier (the leader expects both CTAs' bytes).
+//   warp 1       TMEM allocation (both CTAs, pair-wide) and, in the leader CTA, MMA issue:
+//                4 x tcgen05.mma (K = 32) per slab; tcgen05.commit multicasts stage release and
+//                accumulator-ready signals to both CTAs.
+//   warps 4..11  epilogue: warp w reads TMEM lane quarter (w % 4) (tile rows) and column half
+//                (w - 4) / 4; one row per thread.  Both CTAs' epilogue warps release an
+//                accumulator buffer by arriving on the leader's barrier.
+// Register split: warpgroup 0 drops to 56 registers per thread, the epilogue warpgroups rise to
+// 224 (block-wise keeps a 128-column fp32 running sum per thread).
+// Tiles are visited in bands of 8 pair-rows (2048 tokens) so that the activations and weights in
+// use by all pairs at one time stay resident in L2.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -25,21 +35,23 @@
 
 namespace i8q {
 
-constexpr int GEMM_BM = 128;       // tokens per tile (MMA M)
+constexpr int GEMM_BM = 256;       // tokens per pair tile (MMA M, cta_group::2)
 constexpr int GEMM_BK = 128;       // K per slab (bytes of int8 = one 128B swizzle row)
-constexpr int GEMM_GROUP_M = 16;   // token-blocks per raster band
+constexpr int GEMM_GROUP_M = 8;    // pair-tile rows per raster band
 
 template <int BN>
 struct W8A8Cfg {
-  static constexpr int A_BYTES = GEMM_BM * GEMM_BK;
-  static constexpr int B_BYTES = BN * GEMM_BK;
+  static constexpr int A_BYTES = 128 * GEMM_BK;          // this CTA's 128 token rows
+  static constexpr int B_BYTES = (BN / 2) * GEMM_BK;     // this CTA's BN/2 weight rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN >= 256) ? 4 : 6;
-  static constexpr int TMEM_COLS = 2 * BN;               // two accumulator buffers
-  static constexpr int NUM_THREADS = 256;
+  static constexpr int STAGES = 6;
+  static constexpr int TMEM_COLS = 512;                  // two accumulator buffers of BN columns
+  static constexpr int NUM_THREADS = 384;
+  static constexpr int EPI_WARPS = 8;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
-  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM allocation must be a power of two");
+  static_assert(2 * BN <= TMEM_COLS, "two accumulators must fit in TMEM");
+  static_assert(BN % 32 == 0 && BN <= 256, "MMA N");
 };
 
 struct W8A8Args {
@@ -51,6 +63,87 @@ struct W8A8Args {
   int32_t* dbg;         // channel: [M][N] accumulators; block: [M][N][KB] slab partials
 };
 
+// ------------------------------------------------------------------ pair-wide PTX wrappers ----
+__device__ __forceinline__ uint32_t cta_rank_in_cluster() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA 2-D tile load issued by either CTA of the pair; bytes are counted on the barrier at
+// `bar_cluster` (the leader CTA's).
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster,
+                                                 int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive once on the barrier at the same offset in both CTAs of the pair when all prior MMAs end
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair_self(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// 32 lanes x 32 columns of 32-bit registers -> TMEM
+__device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(
+          taddr),
+      "r"(v)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ------------------------------------------------------------------ helpers -------------------
 __device__ __forceinline__ void gemm_tile_coords(int t, int Mt, int Nt, int& mb, int& nb) {
   const int band_tiles = GEMM_GROUP_M * Nt;
   const int band = t / band_tiles;
@@ -61,10 +154,11 @@ __device__ __forceinline__ void gemm_tile_coords(int t, int Mt, int Nt, int& mb,
   nb = idx / rows;
 }
 
-// Exact int32 -> fp32 for |p| < 2^22: place p in the mantissa of 1.5 * 2^23 and subtract.
-__device__ __forceinline__ float i2f_small_exact(uint32_t p) {
-  return __int_as_float(0x4B400000 + (int)p) - 12582912.0f;
-}
+// fp32 bits 0x4B400000 = 1.5 * 2^23 = 12582912.  An int32 accumulator that starts from these bits
+// holds 0x4B400000 + P after the MMA adds P; for |P| < 2^22 those are exactly the bits of the
+// float 12582912 + P, so subtracting 12582912 recovers P exactly.
+constexpr uint32_t kAccBiasBits = 0x4B400000u;
+constexpr float kAccBias = 12582912.0f;
 
 __device__ __forceinline__ void store_row8(void* y, bool f32out, int64_t off, const float (&v)[8]) {
   if (f32out) {
@@ -86,11 +180,12 @@ __device__ __forceinline__ void store_row8(void* y, bool f32out, int64_t off, co
 }
 
 template <int BN, bool BLOCKWISE, bool OUT_F32, bool DEBUG>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     k_gemm_w8a8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const W8A8Args args) {
   using C = W8A8Cfg<BN>;
-  static_assert(!BLOCKWISE || BN == 128, "block-wise tiles are one weight block wide");
+  static_assert(!BLOCKWISE || BN == 256, "block-wise pair tiles are two weight blocks wide");
+  constexpr int HALF = BN / 2;                 // columns per epilogue warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -104,6 +199,9 @@ __global__ void __launch_bounds__(256, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cta_rank_in_cluster();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int M = args.M, N = args.N, K = args.K;
   const int Mt = (M + GEMM_BM - 1) / GEMM_BM, Nt = (N + BN - 1) / BN, KB = K / GEMM_BK;
   const int num_tiles = Mt * Nt;
@@ -115,7 +213,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);   // one arrival per epilogue warp
+      mbar_init(&tempty[a], 2 * C::EPI_WARPS);   // every epilogue warp of both CTAs
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -126,48 +224,52 @@ __global__ void __launch_bounds__(256, 1)
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+  if (warp < 4) {
+    setmaxnreg_dec<40>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t filled = 0, fill_parity = 0;   // per stage: a load was issued / its phase parity
+      uint32_t expected = 0, exp_parity = 0;   // leader: stages whose completion it expects
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      for (int t = pair; ok && t < num_tiles; t += npairs) {
         int mb, nb;
         gemm_tile_coords(t, Mt, Nt, mb, nb);
+        const int arow = mb * GEMM_BM + (int)rank * 128;
+        const int brow = nb * BN + (int)rank * HALF;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, SITE_EMPTY, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * GEMM_BK, mb * GEMM_BM);
-          tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * GEMM_BK, nb * BN);
-          filled |= 1u << stage;
-          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+          if (leader) {
+            mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+            expected |= 1u << stage;
+            exp_parity = (exp_parity & ~(1u << stage)) | (phase << stage);
+          }
+          const uint32_t bar = map_to_rank(&full[stage], 0);
+          tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, bar, kb * GEMM_BK, arow);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, bar, kb * GEMM_BK, brow);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
-      if (!ok) {  // let every copy already in flight land before the CTA can exit
+      if (!ok && leader) {  // let copies already in flight land before the pair can exit
         for (int s = 0; s < C::STAGES; ++s)
-          if (filled & (1u << s)) mbar_wait(&full[s], (fill_parity >> s) & 1u, SITE_DRAIN, nullptr);
+          if (expected & (1u << s)) mbar_wait(&full[s], (exp_parity >> s) & 1u, SITE_DRAIN, nullptr);
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0 && leader) {
+      // ------------------------------------------------------------------ MMA issuer (leader)
       constexpr uint32_t idesc = idesc_i8(GEMM_BM, BN);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_iter = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+      for (int t = pair; ok && t < num_tiles; t += npairs) {
         uint32_t acc = 0;
         if (!BLOCKWISE) {
           acc = acc_iter & 1;
@@ -176,8 +278,9 @@ __global__ void __launch_bounds__(256, 1)
         }
         for (int kb = 0; kb < KB; ++kb) {
           if (BLOCKWISE) {
+            // use u of buffer acc waits for the epilogue's u-th release (its bias initialisation)
             acc = acc_iter & 1;
-            if (!mbar_wait(&tempty[acc], ((acc_iter >> 1) & 1) ^ 1, SITE_TMEM_EMPTY, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&tempty[acc], (acc_iter >> 1) & 1, SITE_TMEM_EMPTY, abort_flag)) { ok = false; break; }
             tc_fence_after();
           }
           if (!mbar_wait(&full[stage], phase, SITE_FULL, abort_flag)) { ok = false; break; }
@@ -187,35 +290,55 @@ __global__ void __launch_bounds__(256, 1)
           const uint32_t d = tmem + acc * BN;
 #pragma unroll
           for (int kk = 0; kk < GEMM_BK / 32; ++kk) {
-            const uint32_t accumulate = BLOCKWISE ? (kk > 0) : (kb > 0 || kk > 0);
-            mma_i8(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc, accumulate);
+            const uint32_t accumulate = BLOCKWISE ? 1u : (uint32_t)(kb > 0 || kk > 0);
+            mma_i8_pair(d, sw128_kmajor_desc(a0 + kk * 32), sw128_kmajor_desc(b0 + kk * 32), idesc, accumulate);
           }
-          tc_commit(&empty[stage]);
+          tc_commit_pair_both(&empty[stage]);
           if (BLOCKWISE) {
-            tc_commit(&tfull[acc]);
+            tc_commit_pair_both(&tfull[acc]);
             ++acc_iter;
           }
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!BLOCKWISE && ok) {
-          tc_commit(&tfull[acc]);
+          tc_commit_pair_both(&tfull[acc]);
           ++acc_iter;
         }
       }
       // every MMA this thread issued has finished once `done` completes
-      tc_commit(done);
+      tc_commit_pair_self(done);
       mbar_wait(done, 0, SITE_DRAIN, nullptr);
     }
-  } else if (warp >= 4) {
+  } else {
+    setmaxnreg_inc<232>();
     // ------------------------------------------------------------------ epilogue
-    const int q = warp & 3;                        // TMEM lane quarter = tile rows 32q..32q+31
+    const int q = warp & 3;                         // TMEM lane quarter
+    const int h = (warp - 4) >> 2;                  // column half
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const int row = (int)rank * 128 + q * 32 + lane;  // row within the 256-row pair tile
+    const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0), tempty_leader1 = map_to_rank(&tempty[1], 0);
     uint32_t acc_iter = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+
+    if constexpr (BLOCKWISE) {
+      // pre-load both accumulator buffers with the float bias, then release them to the MMA
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int c = 0; c < HALF / 32; ++c) tmem_st32_const(tmem + lane_addr + a * BN + h * HALF + c * 32, kAccBiasBits);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_cluster(tempty_leader0);
+        mbar_arrive_cluster(tempty_leader1);
+      }
+    }
+
+    for (int t = pair; t < num_tiles; t += npairs) {
       int mb, nb;
       gemm_tile_coords(t, Mt, Nt, mb, nb);
-      const int m = mb * GEMM_BM + q * 32 + lane;
-      const int n0 = nb * BN;
+      const int m = mb * GEMM_BM + row;
+      const int n0 = nb * BN + h * HALF;           // first column of this warp's half
       const bool row_ok = m < M;
       if constexpr (!BLOCKWISE) {
         const uint32_t acc = acc_iter & 1;
@@ -223,9 +346,9 @@ __global__ void __launch_bounds__(256, 1)
         tc_fence_after();
         const float sxm = row_ok ? __ldg(args.sx + m) : 0.f;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < HALF / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(tmem + lane_addr + acc * BN + c * 32, r);
+          tmem_ld32(tmem + lane_addr + acc * BN + h * HALF + c * 32, r);
           tmem_ld_wait();
           const int nc = n0 + c * 32;
           if (row_ok) {
@@ -251,56 +374,67 @@ __global__ void __launch_bounds__(256, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[acc]);
+        if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
         ++acc_iter;
       } else {
-        float sum[BN];
+        float2 sum[HALF / 2];
 #pragma unroll
-        for (int j = 0; j < BN; ++j) sum[j] = 0.f;
+        for (int j = 0; j < HALF / 2; ++j) sum[j] = make_float2(0.f, 0.f);
         bool ok = true;
-        const float* swrow = args.sw + (int64_t)nb * KB;   // BN == 128: tile n-block == weight block
+        const bool cols_ok = n0 < N;                    // this weight block exists
+        const float* swrow = args.sw + (int64_t)(n0 / 128) * KB;
         float s_next = 0.f;
-        if (KB > 0 && row_ok) s_next = __ldg(args.sx + m) * __ldg(swrow);
+        if (KB > 0 && row_ok && cols_ok) s_next = __ldg(args.sx + m) * __ldg(swrow);
         for (int kb = 0; kb < KB; ++kb) {
           const float s = s_next;
-          if (kb + 1 < KB && row_ok)
+          if (kb + 1 < KB && row_ok && cols_ok)
             s_next = __ldg(args.sx + (int64_t)(kb + 1) * args.ld_sx + m) * __ldg(swrow + kb + 1);
+          const float2 s2 = make_float2(s, s);
+          const float2 nbias = make_float2(-kAccBias, -kAccBias);
           const uint32_t acc = acc_iter & 1;
           if (!warp_wait(&tfull[acc], (acc_iter >> 1) & 1, SITE_TMEM_FULL, abort_flag)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t base = tmem + lane_addr + acc * BN + h * HALF;
 #pragma unroll
-          for (int c = 0; c < BN / 32; c += 2) {
-            uint32_t r0[32], r1[32];
-            tmem_ld32(tmem + lane_addr + acc * BN + c * 32, r0);
-            tmem_ld32(tmem + lane_addr + acc * BN + (c + 1) * 32, r1);
+          for (int c = 0; c < HALF / 16; ++c) {
+            uint32_t r0[16];
+            tmem_ld16(base + c * 16, r0);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sum[c * 32 + j] = fmaf(i2f_small_exact(r0[j]), s, sum[c * 32 + j]);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) sum[(c + 1) * 32 + j] = fmaf(i2f_small_exact(r1[j]), s, sum[(c + 1) * 32 + j]);
+            for (int j = 0; j < 8; ++j) {
+              const float2 p = __fadd2_rn(make_float2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1])), nbias);
+              sum[c * 8 + j] = __ffma2_rn(p, s2, sum[c * 8 + j]);
+            }
             if constexpr (DEBUG) {
               if (row_ok) {
-                for (int j = 0; j < 32; ++j) {
-                  if (n0 + c * 32 + j < N) args.dbg[((int64_t)m * N + n0 + c * 32 + j) * KB + kb] = (int32_t)r0[j];
-                  if (n0 + (c + 1) * 32 + j < N) args.dbg[((int64_t)m * N + n0 + (c + 1) * 32 + j) * KB + kb] = (int32_t)r1[j];
+                for (int j = 0; j < 16; ++j) {
+                  const int na = n0 + c * 16 + j;
+                  if (na < N) args.dbg[((int64_t)m * N + na) * KB + kb] = (int32_t)(r0[j] - kAccBiasBits);
                 }
               }
             }
           }
+          // re-arm this half of the buffer with the bias for its next use, then release it
+#pragma unroll
+          for (int c = 0; c < HALF / 32; ++c) tmem_st32_const(base + c * 32, kAccBiasBits);
+          tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
+          if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
           ++acc_iter;
         }
         if (!ok) break;
-        if (row_ok) {
+        if (row_ok && cols_ok) {
 #pragma unroll
-          for (int g = 0; g < BN / 8; ++g) {
+          for (int g = 0; g < HALF / 8; ++g) {
             const int n = n0 + g * 8;
             if (n < N) {
               float v[8];
 #pragma unroll
-              for (int j = 0; j < 8; ++j) v[j] = sum[g * 8 + j];
+              for (int j = 0; j < 4; ++j) {
+                v[2 * j] = sum[g * 4 + j].x;
+                v[2 * j + 1] = sum[g * 4 + j].y;
+              }
               store_row8(args.y, OUT_F32, (int64_t)m * N + n, v);
             }
           }
@@ -311,8 +445,9 @@ __global__ void __launch_bounds__(256, 1)
 
   tc_fence_before();
   __syncthreads();
+  cluster_sync();   // neither CTA leaves while its pair may still touch its shared memory / TMEM
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == 1) tmem_dealloc_pair(tmem, C::TMEM_COLS);
 }
 
 }  // namespace i8q

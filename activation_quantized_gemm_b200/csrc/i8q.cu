@@ -197,18 +197,35 @@ static i8q_status gemm_w8a8_common_checks(const int8_t* xq, const float* sx, con
 }
 
 template <int BN, bool BLOCKWISE, bool F32, bool DBG>
-static i8q_status launch_w8a8(const CUtensorMap& ta, const CUtensorMap& tb, const W8A8Args& a, int sms,
-                              cudaStream_t s) {
+static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms, cudaStream_t s) {
   using C = W8A8Cfg<BN>;
   auto kern = k_gemm_w8a8<BN, BLOCKWISE, F32, DBG>;
   static std::once_flag once;
   static i8q_status attr = I8Q_OK;
   std::call_once(once, [&] { attr = set_smem(kern, C::SMEM_BYTES); });
   if (attr) return attr;
+  CUtensorMap ta, tb;
+  i8q_status st = make_tmap_2d(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, a.K, 128, GEMM_BK,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  st = make_tmap_2d(&tb, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, a.K, BN / 2, GEMM_BK,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
   const int64_t tiles = cdiv(a.M, GEMM_BM) * cdiv(a.N, BN);
-  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-  kern<<<grid, C::NUM_THREADS, C::SMEM_BYTES, s>>>(ta, tb, a);
-  I8Q_LAUNCHED("k_gemm_w8a8");
+  const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, a));
   return I8Q_OK;
 }
 
@@ -361,14 +378,9 @@ i8q_status i8q_gemm_w8a8_channel(const int8_t* xq, const float* sx, const int8_t
     return I8Q_OK;
   }
   constexpr int BN = 256;
-  CUtensorMap ta, tb;
-  st = make_tmap_2d(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, GEMM_BM, GEMM_BK, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st) return st;
-  st = make_tmap_2d(&tb, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, BN, GEMM_BK, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st) return st;
   W8A8Args a{sx, 0, sw, (int)M, (int)N, (int)K, y, dbg};
-  if (dbg) return launch_w8a8<BN, false, false, true>(ta, tb, a, sms, S(stream));
-  return launch_w8a8<BN, false, false, false>(ta, tb, a, sms, S(stream));
+  if (dbg) return launch_w8a8<BN, false, false, true>(xq, wq, a, sms, S(stream));
+  return launch_w8a8<BN, false, false, false>(xq, wq, a, sms, S(stream));
 }
 
 i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx, const int8_t* wq, const float* sw,
@@ -386,20 +398,15 @@ i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx,
     I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * osz, S(stream)));
     return I8Q_OK;
   }
-  constexpr int BN = 128;
-  CUtensorMap ta, tb;
-  st = make_tmap_2d(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K, K, GEMM_BM, GEMM_BK, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st) return st;
-  st = make_tmap_2d(&tb, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, BN, GEMM_BK, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (st) return st;
+  constexpr int BN = 256;
   W8A8Args a{sx, ld_sx, sw, (int)M, (int)N, (int)K, y, dbg};
   const bool f32 = out == I8Q_OUT_FP32;
   if (dbg) {
-    if (f32) return launch_w8a8<BN, true, true, true>(ta, tb, a, sms, S(stream));
-    return launch_w8a8<BN, true, false, true>(ta, tb, a, sms, S(stream));
+    if (f32) return launch_w8a8<BN, true, true, true>(xq, wq, a, sms, S(stream));
+    return launch_w8a8<BN, true, false, true>(xq, wq, a, sms, S(stream));
   }
-  if (f32) return launch_w8a8<BN, true, true, false>(ta, tb, a, sms, S(stream));
-  return launch_w8a8<BN, true, false, false>(ta, tb, a, sms, S(stream));
+  if (f32) return launch_w8a8<BN, true, true, false>(xq, wq, a, sms, S(stream));
+  return launch_w8a8<BN, true, false, false>(xq, wq, a, sms, S(stream));
 }
 
 // ---------------------------------------------------------------- a6 -------------------------
