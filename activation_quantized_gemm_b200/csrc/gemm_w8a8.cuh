@@ -79,7 +79,7 @@ __device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
   return r;
 }
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // TMA 2-D tile load issued by either CTA of the pair; bytes are counted on the barrier at
 // `bar_cluster` (the leader CTA's).
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    setmaxnreg_dec<40>();
+    setmaxnreg_dec<24>();
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------------ TMA producer
       int stage = 0;
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait(done, 0, SITE_DRAIN, nullptr);
     }
   } else {
-    setmaxnreg_inc<232>();
+    setmaxnreg_inc<240>();
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;                         // TMEM lane quarter
     const int h = (warp - 4) >> 2;                  // column half
@@ -381,42 +381,47 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int j = 0; j < HALF / 2; ++j) sum[j] = make_float2(0.f, 0.f);
         bool ok = true;
-        const bool cols_ok = n0 < N;                    // this weight block exists
+        const bool live = row_ok && n0 < N;              // this row and weight block exist
         const float* swrow = args.sw + (int64_t)(n0 / 128) * KB;
-        float s_next = 0.f;
-        if (KB > 0 && row_ok && cols_ok) s_next = __ldg(args.sx + m) * __ldg(swrow);
+        // raw scales of the next slab are loaded one slab ahead; the product is formed when used
+        float sx_next = 0.f, sw_next = 0.f;
+        if (KB > 0 && live) {
+          sx_next = __ldg(args.sx + m);
+          sw_next = __ldg(swrow);
+        }
+        const float2 nbias = make_float2(-kAccBias, -kAccBias);
         for (int kb = 0; kb < KB; ++kb) {
-          const float s = s_next;
-          if (kb + 1 < KB && row_ok && cols_ok)
-            s_next = __ldg(args.sx + (int64_t)(kb + 1) * args.ld_sx + m) * __ldg(swrow + kb + 1);
+          const float s = sx_next * sw_next;
+          if (kb + 1 < KB && live) {
+            sx_next = __ldg(args.sx + (int64_t)(kb + 1) * args.ld_sx + m);
+            sw_next = __ldg(swrow + kb + 1);
+          }
           const float2 s2 = make_float2(s, s);
-          const float2 nbias = make_float2(-kAccBias, -kAccBias);
           const uint32_t acc = acc_iter & 1;
           if (!warp_wait(&tfull[acc], (acc_iter >> 1) & 1, SITE_TMEM_FULL, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t base = tmem + lane_addr + acc * BN + h * HALF;
 #pragma unroll
-          for (int c = 0; c < HALF / 16; ++c) {
-            uint32_t r0[16];
-            tmem_ld16(base + c * 16, r0);
+          for (int c = 0; c < HALF / 32; ++c) {
+            uint32_t r0[32];
+            tmem_ld32(base + c * 32, r0);
             tmem_ld_wait();
+            // re-arm these columns with the bias for the buffer's next use while the math runs
+            tmem_st32_const(base + c * 32, kAccBiasBits);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 16; ++j) {
               const float2 p = __fadd2_rn(make_float2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1])), nbias);
-              sum[c * 8 + j] = __ffma2_rn(p, s2, sum[c * 8 + j]);
+              sum[c * 16 + j] = __ffma2_rn(p, s2, sum[c * 16 + j]);
             }
             if constexpr (DEBUG) {
               if (row_ok) {
-                for (int j = 0; j < 16; ++j) {
-                  const int na = n0 + c * 16 + j;
+                for (int j = 0; j < 32; ++j) {
+                  const int na = n0 + c * 32 + j;
                   if (na < N) args.dbg[((int64_t)m * N + na) * KB + kb] = (int32_t)(r0[j] - kAccBiasBits);
                 }
               }
             }
           }
-          // re-arm this half of the buffer with the bias for its next use, then release it
-#pragma unroll
-          for (int c = 0; c < HALF / 32; ++c) tmem_st32_const(base + c * 32, kAccBiasBits);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
@@ -424,7 +429,7 @@ __global__ void __launch_bounds__(384, 1)
           ++acc_iter;
         }
         if (!ok) break;
-        if (row_ok && cols_ok) {
+        if (live) {
 #pragma unroll
           for (int g = 0; g < HALF / 8; ++g) {
             const int n = n0 + g * 8;
