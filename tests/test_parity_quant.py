@@ -126,3 +126,66 @@ def test_requant_fp8_channel(q, N, K):
 
 def test_status_check_clean(q):
     q.i8q_status_check()
+
+
+def _reciprocal_traps(n_scales=400, seed=21):
+    """bf16 groups in which x * fp32(1/s) and the true quotient x / s round to different codes.
+
+    For random bf16 absmax values a, every positive bf16 x <= a is tried; the ones where the
+    reciprocal product lands on the other side of a half-integer (or on a tie the quotient does
+    not reach) are collected, and each group is [a, traps..., random fill <= a], with random signs.
+    """
+    rng = np.random.default_rng(seed)
+    all_pos = (np.arange(1, 0x7F80, dtype=np.uint32) << 16).view(np.float32)     # positive finite bf16
+    rows = []
+    for _ in range(n_scales):
+        a = np.float32(all_pos[rng.integers(0x3000, 0x5000)])                       # ~1e-5 .. 1e10
+        s = np.float32(a / np.float32(127))
+        xs = all_pos[all_pos <= a]
+        q_div = np.rint(xs / s)
+        q_rec = np.rint(xs * (np.float32(1) / s))
+        traps = xs[q_div != q_rec]
+        if traps.size == 0:
+            continue
+        row = np.empty(128, np.float32)
+        row[0] = a
+        k = min(traps.size, 100)
+        row[1:1 + k] = rng.choice(traps, k, replace=False)
+        row[1 + k:] = rng.choice(xs, 127 - k)
+        row[1:] *= np.where(rng.random(127) < 0.5, -1, 1).astype(np.float32)
+        rows.append(row)
+    assert len(rows) >= 50, len(rows)
+    return O.f32_to_bf16_rne(np.stack(rows))
+
+
+def test_quantizer_reciprocal_traps(q):
+    x = _reciprocal_traps()
+    M = x.shape[0]
+    xq_ref, sx_ref = O.quant_act_token_group(x)
+    xq = empty((M, 128), torch.int8)
+    sx = empty((1, (M + 3) // 4 * 4), torch.float32)
+    q.i8q_quant_act_token_group(dev(x), xq, sx)
+    xq2 = empty((M, 128), torch.int8)
+    sx2 = empty((M,), torch.float32)
+    q.i8q_quant_act_token(dev(x), xq2, sx2)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(xq), xq_ref) and np.array_equal(host(sx)[0, :M], sx_ref[:, 0])
+    assert np.array_equal(host(xq2), xq_ref) and np.array_equal(host(sx2), sx_ref[:, 0])
+
+
+def test_quantizer_random_magnitudes(q):
+    """4M elements: each 128-group has a random bf16 absmax (1e-30 .. 1e30) and uniform codes below it."""
+    rng = np.random.default_rng(22)
+    G = 32768
+    e = rng.uniform(-100, 100, G)
+    a = (2.0 ** e).astype(np.float32)
+    v = (rng.uniform(-1, 1, (G, 128)) * a[:, None]).astype(np.float32)
+    v[np.arange(G), rng.integers(0, 128, G)] = a * np.where(rng.random(G) < 0.5, -1, 1)
+    x = O.f32_to_bf16_rne(v).reshape(1024, 32 * 128)
+    xq_ref, sx_ref = O.quant_act_token_group(x)
+    xq = empty(x.shape, torch.int8)
+    sx = empty((32, 1024), torch.float32)
+    q.i8q_quant_act_token_group(dev(x), xq, sx)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(xq), xq_ref)
+    assert np.array_equal(host(sx).T, sx_ref)
