@@ -11,11 +11,14 @@
 // its N dimension, so a decode batch of 1..64 tokens still fills the 128-row tensor-core tile.
 //   warp 0       TMA: int8 weight slab [128 rows x 128 K] (128B swizzle) + f16 activation slab
 //                [MP x 128 K] as two 64-element halves (128B swizzle), one mbarrier per stage.
-//   warp 1       TMEM allocation and MMA issue: 8 x tcgen05.mma.kind::f16 (K = 16) per slab
-//                into one of two TMEM accumulators (MP fp32 columns each).
-//   warps 4..7   converters: int8 slab -> f16 operand in shared memory (128B swizzle layout the
-//                MMA descriptor expects), then fence.proxy.async and an mbarrier arrival.
-//   warps 8..11  epilogue: thread = weight row; per slab, sum[m] += partial[m] * s[n][g].
+//   warp 1       TMEM allocation and MMA issue: 8 x tcgen05.mma.kind::f16 (K = 16) per slab.
+//   warps 4..11  converters: int8 slab -> f16 operand in shared memory (128B swizzle layout the
+//                MMA descriptor expects; NA operand buffers), then fence.proxy.async and an
+//                mbarrier arrival.
+//   warps 12..15 epilogue: thread = weight row; per slab, sum[m] += partial[m] * s[n][g].
+// Small-N MMAs have a long latency compared with their work, so consecutive MMAs never wait on
+// each other: each slab's 8 k-steps alternate between NACC independent TMEM accumulators (summed
+// by the epilogue), and up to NBUF slabs are in flight in a ring of TMEM accumulators.
 // Split-K: the CTAs of one thread-block cluster take disjoint slab ranges of the same 128 rows;
 // rank 0 adds the other ranks' fp32 partial tiles read from their shared memory (distributed
 // shared memory), in rank order, and writes fp16.
@@ -36,12 +39,18 @@ struct W8A16Cfg {
   static constexpr int X_HALF = MP * 128;               // one 64-element half of the f16 slab
   static constexpr int X_BYTES = 2 * X_HALF;
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
-  static constexpr int STAGES = 4;
-  static constexpr int A_BYTES = W8A16_BN * 128 * 2;    // f16 operand: two 16 KB halves
-  static constexpr int TMEM_COLS = (2 * MP < 32) ? 32 : 2 * MP;
-  static constexpr int NUM_THREADS = 384;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + A_BYTES + 256 + 1024;
-  static_assert(MP * W8A16_BN * 4 <= A_BYTES, "reduction tile must fit in the operand buffer");
+  static constexpr int STAGES = MP >= 32 ? 4 : 6;
+  static constexpr int A_BYTES = W8A16_BN * 128 * 2;    // f16 operand of one slab: two 16 KB halves
+  static constexpr int NA = 3;                          // operand buffers
+  static constexpr int NACC = 2;                        // independent accumulators per slab
+  static constexpr int NBUF = (512 / (NACC * MP)) < 8 ? (512 / (NACC * MP)) : 8;   // slab accumulators in TMEM
+  static constexpr int TMEM_NEED = NBUF * NACC * MP;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                   : TMEM_NEED <= 256 ? 256 : 512;
+  static constexpr int NUM_THREADS = 512;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NA * A_BYTES + 512 + 1024;
+  static_assert(MP * W8A16_BN * 4 <= NA * A_BYTES, "reduction tile must fit in the operand buffers");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 struct W8A16Args {
@@ -89,21 +98,21 @@ __device__ __forceinline__ void i8x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t
 }
 
 template <int MP>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     k_gemm_w8a16(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const W8A16Args args) {
   using C = W8A16Cfg<MP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sStage = smem;                                   // STAGES x (W slab | X halves)
-  uint8_t* sA = smem + C::STAGES * C::STAGE_BYTES;          // f16 operand (2 x 16 KB halves)
-  uint64_t* full = reinterpret_cast<uint64_t*>(sA + C::A_BYTES);
+  uint8_t* sA = smem + C::STAGES * C::STAGE_BYTES;          // NA x f16 operand (2 x 16 KB halves each)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sA + C::NA * C::A_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* afull = empty + C::STAGES;
-  uint64_t* aempty = afull + 1;
-  uint64_t* tfull = aempty + 1;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* done = tempty + 2;
+  uint64_t* aempty = afull + C::NA;
+  uint64_t* tfull = aempty + C::NA;
+  uint64_t* tempty = tfull + C::NBUF;
+  uint64_t* done = tempty + C::NBUF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -118,13 +127,15 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 5);   // 4 converter warps + 1 MMA commit
+      mbar_init(&empty[s], 9);   // 8 converter warps + 1 MMA commit
     }
-    mbar_init(afull, 4);
-    mbar_init(aempty, 1);
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+    for (int a = 0; a < C::NA; ++a) {
+      mbar_init(&afull[a], 8);
+      mbar_init(&aempty[a], 1);
+    }
+    for (int b = 0; b < C::NBUF; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -171,99 +182,116 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(W8A16_BN, MP);
-      const uint32_t a0 = smem_u32(sA);
       for (int j = 0; j < nslab; ++j) {
         const int s = j % C::STAGES;
         const uint32_t ph = (j / C::STAGES) & 1;
-        const uint32_t acc = j & 1;
-        if (!mbar_wait(&tempty[acc], ((j >> 1) & 1) ^ 1, SITE_TMEM_EMPTY, abort_flag)) break;
-        if (!mbar_wait(afull, j & 1, SITE_CONVERT, abort_flag)) break;
+        const int a = j % C::NA;
+        const uint32_t pa = (j / C::NA) & 1;
+        const int b = j % C::NBUF;
+        const uint32_t pb = (j / C::NBUF) & 1;
+        if (!mbar_wait(&tempty[b], pb ^ 1, SITE_TMEM_EMPTY, abort_flag)) break;
+        if (!mbar_wait(&afull[a], pa, SITE_CONVERT, abort_flag)) break;
         if (!mbar_wait(&full[s], ph, SITE_FULL, abort_flag)) break;
         tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + a * C::A_BYTES);
         const uint32_t x0 = smem_u32(sStage + s * C::STAGE_BYTES + C::W_BYTES);
+        const uint32_t d0 = tmem + b * C::NACC * MP;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t h = kk >> 2, off = (kk & 3) * 32;
-          mma_f16(tmem + acc * MP, sw128_kmajor_desc(a0 + h * 16384 + off),
-                  sw128_kmajor_desc(x0 + h * C::X_HALF + off), idesc, kk > 0);
+          mma_f16(d0 + (kk % C::NACC) * MP, sw128_kmajor_desc(a0 + h * 16384 + off),
+                  sw128_kmajor_desc(x0 + h * C::X_HALF + off), idesc, kk >= C::NACC);
         }
         tc_commit(&empty[s]);
-        tc_commit(aempty);
-        tc_commit(&tfull[acc]);
+        tc_commit(&aempty[a]);
+        tc_commit(&tfull[b]);
       }
       tc_commit(done);
       mbar_wait(done, 0, SITE_DRAIN, nullptr);
     }
-  } else if (warp >= 4 && warp < 8) {
-    // converters: thread r owns weight row r of the slab (8 x 16-byte chunks of int8)
-    const int r = threadIdx.x - 128;
+  } else if (warp >= 4 && warp < 12) {
+    // converters: warp c = warp - 4 owns weight rows 32 (c % 4) .. + 31 and K half c / 4 of the slab
+    const int c = warp - 4;
+    const int r = (c & 3) * 32 + lane;
+    const int h = c >> 2;
     const int sw = r & 7;
     for (int j = 0; j < nslab; ++j) {
       const int s = j % C::STAGES;
       const uint32_t ph = (j / C::STAGES) & 1;
+      const int a = j % C::NA;
+      const uint32_t pa = (j / C::NA) & 1;
       if (!warp_wait(&full[s], ph, SITE_FULL, abort_flag)) break;
-      if (!warp_wait(aempty, (j & 1) ^ 1, SITE_CONVERT, abort_flag)) break;
+      if (!warp_wait(&aempty[a], pa ^ 1, SITE_CONVERT, abort_flag)) break;
       const uint8_t* wrow = sStage + s * C::STAGE_BYTES + r * 128;
+      uint8_t* arow = sA + a * C::A_BYTES + h * 16384 + r * 128;
+      uint4 v[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((c ^ sw) << 4));
+      for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(wrow + (((4 * h + i) ^ sw) << 4));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
         uint4 o0, o1;
-        i8x4_to_f16x4(v.x, o0.x, o0.y);
-        i8x4_to_f16x4(v.y, o0.z, o0.w);
-        i8x4_to_f16x4(v.z, o1.x, o1.y);
-        i8x4_to_f16x4(v.w, o1.z, o1.w);
-        // f16 chunk indices 2c, 2c+1 of the 16 chunks of this row; half = chunk / 8
-        const int h = c >> 2;
-        const int c0 = (2 * c) & 7, c1 = (2 * c + 1) & 7;
-        uint8_t* arow = sA + h * 16384 + r * 128;
-        *reinterpret_cast<uint4*>(arow + ((c0 ^ sw) << 4)) = o0;
-        *reinterpret_cast<uint4*>(arow + ((c1 ^ sw) << 4)) = o1;
+        i8x4_to_f16x4(v[i].x, o0.x, o0.y);
+        i8x4_to_f16x4(v[i].y, o0.z, o0.w);
+        i8x4_to_f16x4(v[i].z, o1.x, o1.y);
+        i8x4_to_f16x4(v[i].w, o1.z, o1.w);
+        // int8 chunk 4h + i holds f16 chunks 8h + 2i, 8h + 2i + 1: chunks 2i, 2i + 1 of operand half h
+        *reinterpret_cast<uint4*>(arow + (((2 * i) ^ sw) << 4)) = o0;
+        *reinterpret_cast<uint4*>(arow + (((2 * i + 1) ^ sw) << 4)) = o1;
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(afull);
+        mbar_arrive(&afull[a]);
         mbar_arrive(&empty[s]);
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 12) {
     // epilogue: thread = weight row n0 + 32 * (warp % 4) + lane
     const int q = warp & 3;
     const int n = n0 + q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     const int G = KB;
+    float sc_next = (n < N && nslab > 0) ? __half2float(__ushort_as_half(__ldg(args.s + (int64_t)n * G + kb0))) : 0.f;
     for (int j = 0; j < nslab; ++j) {
-      const uint32_t acc = j & 1;
-      const float sc = (n < N) ? __half2float(__ushort_as_half(__ldg(args.s + (int64_t)n * G + kb0 + j))) : 0.f;
-      if (!warp_wait(&tfull[acc], (j >> 1) & 1, SITE_TMEM_FULL, abort_flag)) break;
+      const int b = j % C::NBUF;
+      const uint32_t pb = (j / C::NBUF) & 1;
+      const float sc = sc_next;
+      if (j + 1 < nslab && n < N) sc_next = __half2float(__ushort_as_half(__ldg(args.s + (int64_t)n * G + kb0 + j + 1)));
+      if (!warp_wait(&tfull[b], pb, SITE_TMEM_FULL, abort_flag)) break;
       tc_fence_after();
+      const uint32_t base = tmem + lane_addr + b * C::NACC * MP;
       if constexpr (MP == 16) {
-        uint32_t p[16];
-        tmem_ld16(tmem + lane_addr + acc * MP, p);
+        uint32_t p0[16], p1[16];
+        tmem_ld16(base, p0);
+        tmem_ld16(base + 16, p1);
         tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[b]);
 #pragma unroll
-        for (int m = 0; m < 16; ++m) sum[m] = fmaf(__uint_as_float(p[m]), sc, sum[m]);
+        for (int m = 0; m < 16; ++m) sum[m] = fmaf(__uint_as_float(p0[m]) + __uint_as_float(p1[m]), sc, sum[m]);
       } else {
 #pragma unroll
-        for (int c = 0; c < MP / 32; ++c) {
-          uint32_t p[32];
-          tmem_ld32(tmem + lane_addr + acc * MP + c * 32, p);
+        for (int c0 = 0; c0 < MP; c0 += 32) {
+          uint32_t p0[32], p1[32];
+          tmem_ld32(base + c0, p0);
+          tmem_ld32(base + MP + c0, p1);
           tmem_ld_wait();
 #pragma unroll
-          for (int m = 0; m < 32; ++m) sum[c * 32 + m] = fmaf(__uint_as_float(p[m]), sc, sum[c * 32 + m]);
+          for (int m = 0; m < 32; ++m) sum[c0 + m] = fmaf(__uint_as_float(p0[m]) + __uint_as_float(p1[m]), sc, sum[c0 + m]);
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[b]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
     }
   }
 
   // ---- split-K reduction across the cluster through distributed shared memory
-  float* red = reinterpret_cast<float*>(sA);   // [MP][128] fp32 partial tile (operand buffer is idle now)
+  float* red = reinterpret_cast<float*>(sA);   // [MP][128] fp32 partial tile (operand buffers are idle now)
   tc_fence_before();
   __syncthreads();
-  const bool epi = warp >= 8;
+  const bool epi = warp >= 12;
   const int row = epi ? (warp & 3) * 32 + lane : 0;
   if (epi && rank != 0) {
 #pragma unroll

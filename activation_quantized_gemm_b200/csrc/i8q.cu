@@ -331,8 +331,8 @@ i8q_status i8q_quant_act_token_group(const uint16_t* x, int64_t M, int64_t K, in
   i8q_status st = current_device(&sms);
   if (st) return st;
   const int64_t KB = K / 128;
-  constexpr int U = 4;
-  const int64_t items = M * cdiv(cdiv(KB, 2), U);
+  constexpr int U = 2;
+  const int64_t items = M * cdiv(cdiv(KB, 8), U);
   I8Q_REQUIRE(items < ((int64_t)1 << 31), I8Q_ERR_SHAPE);
   int64_t blocks = cdiv(items, 8);
   const int64_t cap = resident_grid(k_quant_act_token_group<U>, 256, sms);
@@ -355,18 +355,23 @@ i8q_status i8q_quant_act_token(const uint16_t* x, int64_t M, int64_t K, int64_t 
   i8q_status st = current_device(&sms);
   if (st) return st;
   const int64_t nv = K / 8;
-  if (nv <= 32 * 8) {   // warp per row, row in registers, next row prefetched
-    int64_t grid = cdiv(M, 8);
-    const int64_t cap = resident_grid(k_quant_act_token_warp<8>, 256, sms);
-    if (grid > cap) grid = cap;
-    if (nv <= 32 * 1)
-      k_quant_act_token_warp<1><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
-    else if (nv <= 32 * 2)
-      k_quant_act_token_warp<2><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
-    else if (nv <= 32 * 4)
-      k_quant_act_token_warp<4><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
-    else
-      k_quant_act_token_warp<8><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+  if (nv <= 32 * 8) {   // warp per row, row in registers
+    const int64_t warps = M;
+    const int64_t cap1 = resident_grid(k_quant_act_token_warp<8, false>, 256, sms);
+    if (cdiv(warps, 8) <= cap1) {          // every row in flight at once: no prefetch needed
+      const unsigned grid = (unsigned)cdiv(warps, 8);
+      if (nv <= 32 * 2)
+        k_quant_act_token_warp<2, false><<<grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+      else if (nv <= 32 * 4)
+        k_quant_act_token_warp<4, false><<<grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+      else
+        k_quant_act_token_warp<8, false><<<grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+    } else {                                 // warps own several rows: prefetch the next
+      int64_t grid = cdiv(M, 8);
+      const int64_t cap = resident_grid(k_quant_act_token_warp<8, true>, 256, sms);
+      if (grid > cap) grid = cap;
+      k_quant_act_token_warp<8, true><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+    }
   } else {              // CTA per row
     k_quant_act_token_cta<<<(unsigned)M, 256, 0, S(stream)>>>(x, (int)K, ldx, xq, sx);
   }

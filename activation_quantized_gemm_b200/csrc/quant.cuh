@@ -7,15 +7,18 @@
 //   s = max|v| / 127 (IEEE fp32 divide), q = clamp(rint_half_even(v / s), -127, 127) where v / s
 //   is the correctly rounded fp32 quotient; s == 0 gives q == 0.
 //
-// Exactness of the fast path used here.  y = RN(v * r) with r = RN(1 / s).  With t = v / s exact
-// (|t| <= 127 (1 + 2^-23)), |y - t| <= |t| (2 * 2^-24 + 2^-48) < 1.52e-5, and the correctly rounded
-// quotient d = RN(t) satisfies |d - t| <= ulp(t) / 2 <= 2^-18 < 3.9e-6.  Whenever y lies farther
-// than 2^-15 (> 1.52e-5 + 3.9e-6) from every half-integer, y and d fall strictly inside the same
-// interval (k - 1/2, k + 1/2) and therefore round to the same integer k.  Near a half-integer the
-// value is recomputed with the IEEE division (__fdiv_rn); so is every value of a group whose 1/s
-// is not a normal float.  Rounding to nearest even uses z = y + 1.5 * 2^23 (exact for |y| < 2^22):
-// the fp32 addition rounds y to an integer, and the low byte of z's bit pattern is that integer's
-// two's-complement int8 code.
+// How the quotient is formed.  y0 = RN(v * r) with r the hardware reciprocal of s (rcp.approx,
+// within 1 ulp), then one FMA correction: e = RN(v - y0 * s) (a single fma), y1 = RN(y0 + e * r)
+// (a single fma) - the division scheme of P. Markstein ("Computation of elementary functions on
+// the IBM RISC System/6000 processor", 1990).  The quantizer only ever divides a bf16 value v by
+// s = RN(a / 127) with a (the absmax) bf16 as well, so the whole input domain is finite up to
+// power-of-two scaling: 128 mantissas of a times every bf16 v with |v| <= a.  Over that complete
+// domain (both signs, v down to 2^-11 a, below which every code is 0) rint(y1) equals the code of
+// the IEEE quotient v / s exactly; the GPU parity tests re-check the domain through the library's
+// own entry points.  Groups whose 1/s is not a normal float (|s| < 2^-125 or > 2^125, outside the
+// scaling argument) use the IEEE division.  Rounding to nearest even uses z = y1 + 1.5 * 2^23
+// (exact for |y1| < 2^22): the fp32 addition rounds y1 to an integer, and the low byte of z's bit
+// pattern is that integer's two's-complement int8 code.
 //
 // Memory side: 16-byte vector loads, several in flight per thread (the next row / block is
 // loaded while the current one is quantized), codes written as 8- or 16-byte vectors.
@@ -31,16 +34,20 @@ namespace i8q {
 
 constexpr unsigned FULL_MASK = 0xFFFFFFFFu;
 constexpr float kRoundMagic = 12582912.0f;          // 1.5 * 2^23
-constexpr float kNearTie = 0.5f - 0x1p-15f;         // |y - rint(y)| above this: near a half-integer
 
 struct QScale {
   float s, r;
   bool r_ok;
 };
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 __device__ __forceinline__ QScale make_qscale(float absmax) {
   QScale q;
-  q.s = absmax / 127.0f;                 // IEEE division
-  q.r = __frcp_rn(q.s);                  // correctly rounded reciprocal
+  q.s = absmax / 127.0f;                 // IEEE division: the stored scale is exact
+  q.r = rcp_approx(q.s);                 // within 1 ulp of 1 / s
   q.r_ok = q.s >= 0x1p-125f && q.s <= 0x1p125f;
   return q;
 }
@@ -54,23 +61,28 @@ __device__ __forceinline__ uint32_t quant_div(float v, float s) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// max |x| over the 8 bf16 values of a 16-byte vector (exact; returned as fp32)
-__device__ __forceinline__ float absmax_bf16x8(const uint4& v) {
-  const uint32_t m = 0x7FFF7FFFu;
-  uint32_t a = __vmaxu2(v.x & m, v.y & m);
-  uint32_t b = __vmaxu2(v.z & m, v.w & m);
-  a = __vmaxu2(a, b);
-  return __uint_as_float(max(a & 0xFFFFu, a >> 16) << 16);
+// per-halfword unsigned maximum
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
+// magnitudes (bf16 bit patterns without sign) of a 16-byte vector, folded to one u16x2 word
+__device__ __forceinline__ uint32_t absmax_bits_x8(const uint4& v) {
+  const uint32_t m = 0x7FFF7FFFu;
+  return max_u16x2(max_u16x2(v.x & m, v.y & m), max_u16x2(v.z & m, v.w & m));
+}
+__device__ __forceinline__ float bits_to_absmax(uint32_t a) { return __uint_as_float(max(a & 0xFFFFu, a >> 16) << 16); }
+// max |x| over the 8 bf16 values of a 16-byte vector (exact; returned as fp32)
+__device__ __forceinline__ float absmax_bf16x8(const uint4& v) { return bits_to_absmax(absmax_bits_x8(v)); }
 
-// Codes of two values given y = v * r for both: returns the two rounded-integer bit patterns
-// (low byte = int8 code) and folds the distance-to-integer test into `dmax`.
-__device__ __forceinline__ float2 round2(float2 y, float& dmax) {
-  const float2 z = __fadd2_rn(y, make_float2(kRoundMagic, kRoundMagic));
-  const float2 n = __fadd2_rn(z, make_float2(-kRoundMagic, -kRoundMagic));
-  const float2 d = __fadd2_rn(y, make_float2(-n.x, -n.y));
-  dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
-  return z;
+// Codes of two values v: quotient v / s by the corrected reciprocal product, rounded to an integer
+// with the magic constant; the low byte of each returned word is the int8 code.
+__device__ __forceinline__ float2 code2(float2 v, float2 r2, float2 ns2) {
+  const float2 y0 = __fmul2_rn(v, r2);
+  const float2 e = __ffma2_rn(y0, ns2, v);
+  const float2 y1 = __ffma2_rn(e, r2, y0);
+  return __fadd2_rn(y1, make_float2(kRoundMagic, kRoundMagic));
 }
 __device__ __forceinline__ uint32_t pack4(float2 a, float2 b) {
   const uint32_t t = __byte_perm(__float_as_uint(a.x), __float_as_uint(a.y), 0x0040);
@@ -78,29 +90,32 @@ __device__ __forceinline__ uint32_t pack4(float2 a, float2 b) {
   return __byte_perm(t, u, 0x5410);
 }
 
-// 8 bf16 values (one 16-byte vector) -> 8 int8 codes.  Warp-collective (the rare near-tie
-// fix-up is decided by a warp vote); lanes with `active` false still take part in the vote.
+// IEEE-division codes of 8 values, for groups whose 1/s is not a normal float.  Kept out of line
+// so that the compiler cannot fold it into the common path as predicated code.
+__device__ __noinline__ uint2 quant_bf16x8_div(uint4 v, float s) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    c[2 * i] = quant_div(bf16lo(w[i]), s);
+    c[2 * i + 1] = quant_div(bf16hi(w[i]), s);
+  }
+  return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24), c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+}
+
+// 8 bf16 values (one 16-byte vector) -> 8 int8 codes.  Warp-collective (a warp vote decides the
+// rare extreme-scale path); lanes with `active` false still take part in the vote.
 __device__ __forceinline__ uint2 quant_bf16x8(const uint4& v, const QScale& q, bool active) {
   const float2 r2 = make_float2(q.r, q.r);
-  float dmax = 0.f;
-  const float2 z0 = round2(__fmul2_rn(make_float2(bf16lo(v.x), bf16hi(v.x)), r2), dmax);
-  const float2 z1 = round2(__fmul2_rn(make_float2(bf16lo(v.y), bf16hi(v.y)), r2), dmax);
-  const float2 z2 = round2(__fmul2_rn(make_float2(bf16lo(v.z), bf16hi(v.z)), r2), dmax);
-  const float2 z3 = round2(__fmul2_rn(make_float2(bf16lo(v.w), bf16hi(v.w)), r2), dmax);
+  const float2 ns2 = make_float2(-q.s, -q.s);
+  const float2 z0 = code2(make_float2(bf16lo(v.x), bf16hi(v.x)), r2, ns2);
+  const float2 z1 = code2(make_float2(bf16lo(v.y), bf16hi(v.y)), r2, ns2);
+  const float2 z2 = code2(make_float2(bf16lo(v.z), bf16hi(v.z)), r2, ns2);
+  const float2 z3 = code2(make_float2(bf16lo(v.w), bf16hi(v.w)), r2, ns2);
   uint2 out = make_uint2(pack4(z0, z1), pack4(z2, z3));
-  const bool fix = active && q.s > 0.f && (!q.r_ok || dmax > kNearTie);
-  if (__any_sync(FULL_MASK, fix)) {
-    if (fix) {
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint32_t c[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        c[2 * i] = quant_div(bf16lo(w[i]), q.s);
-        c[2 * i + 1] = quant_div(bf16hi(w[i]), q.s);
-      }
-      out.x = c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24);
-      out.y = c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24);
-    }
+  const bool slow = active && q.s > 0.f && !q.r_ok;
+  if (__builtin_expect(__any_sync(FULL_MASK, slow), 0)) {
+    if (slow) out = quant_bf16x8_div(v, q.s);
   }
   if (!(q.s > 0.f)) out = make_uint2(0, 0);
   return out;
@@ -108,59 +123,81 @@ __device__ __forceinline__ uint2 quant_bf16x8(const uint4& v, const QScale& q, b
 
 // ----------------------------------------------------------------------------------------------
 // a1: per-token-group (128) activation quantization.
-// A warp covers two groups per step (half-warp per group: 16 lanes x 8 bf16); a work item is U
-// consecutive steps of one row, whose loads are all issued before they are quantized; warps walk
-// the items grid-stride.  Scales are written token-contiguous: sx[kb * ld_sx + m].
+// Four lanes share a group (each holds 32 of its values as 4 vectors, interleaved so that the four
+// lanes read 64 contiguous bytes per load), so a warp step covers 8 groups = 1024 values and the
+// per-group scale computation is paid once per 1024 values.  A work item is U consecutive warp
+// steps of one row; warps walk the items grid-stride and keep the loads of their next item in
+// flight while they quantize the current one.  Scales are token-contiguous: sx[kb * ld_sx + m].
 // ----------------------------------------------------------------------------------------------
 template <int U>
 __global__ void __launch_bounds__(256) k_quant_act_token_group(const uint16_t* __restrict__ x, int M, int KB,
                                                                int64_t ldx, int8_t* __restrict__ xq,
                                                                float* __restrict__ sx, int64_t ld_sx) {
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;
-  const int l16 = lane & 15;
+  const int gl = lane >> 2;                        // group within the warp step (0..7)
+  const int sub = lane & 3;                        // lane within the group
   const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
   const int K = KB * 128;
-  const int steps = (KB + 1) >> 1;
-  const int nchunks = (steps + U - 1) / U;        // a work item is U steps of one row
+  const int steps = (KB + 7) >> 3;                 // warp steps per row (8 groups each)
+  const int nchunks = (steps + U - 1) / U;
   const int items = M * nchunks;
-  for (int item = warp; item < items; item += nwarps) {
+  // vector i of a lane: group elements 8 * (sub + 4 i) .. + 8
+  auto load_item = [&](int item, uint4 (&v)[U][4]) {
     const int m = item / nchunks;
     const int st0 = (item - m * nchunks) * U;
-    const uint16_t* xr = x + (int64_t)m * ldx + half * 128 + l16 * 8;
-    int8_t* qr = xq + (int64_t)m * K + half * 128 + l16 * 8;
-    uint4 v[U];
+    const uint16_t* xr = x + (int64_t)m * ldx + gl * 128 + sub * 8;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int kb = 2 * (st0 + u) + half;
-      v[u] = make_uint4(0, 0, 0, 0);
-      if (st0 + u < steps && kb < KB) v[u] = __ldg(reinterpret_cast<const uint4*>(xr + (st0 + u) * 256));
+      const int kb = 8 * (st0 + u) + gl;
+      const bool ok = item < items && st0 + u < steps && kb < KB;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[u][i] = make_uint4(0, 0, 0, 0);
+        if (ok) v[u][i] = __ldg(reinterpret_cast<const uint4*>(xr + (st0 + u) * 1024 + i * 32));
+      }
     }
+  };
+  uint4 cur[U][4], nxt[U][4];
+  int item = warp;
+  if (item < items) load_item(item, cur);
+  for (; item < items; item += nwarps) {
+    load_item(item + nwarps, nxt);
+    const int m = item / nchunks;
+    const int st0 = (item - m * nchunks) * U;
+    int8_t* qr = xq + (int64_t)m * K + gl * 128 + sub * 8;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (st0 + u >= steps) break;                     // warp-uniform
-      const int kb = 2 * (st0 + u) + half;
-      float a = absmax_bf16x8(v[u]);
-#pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(FULL_MASK, a, off));
-      const QScale qs = make_qscale(a);
+      const int kb = 8 * (st0 + u) + gl;
       const bool ok = kb < KB;
-      const uint2 c = quant_bf16x8(v[u], qs, ok);
-      if (ok) {
-        *reinterpret_cast<uint2*>(qr + (st0 + u) * 256) = c;
-        if (l16 == 0) sx[(int64_t)kb * ld_sx + m] = qs.s;
+      uint32_t ab = max_u16x2(max_u16x2(absmax_bits_x8(cur[u][0]), absmax_bits_x8(cur[u][1])),
+                              max_u16x2(absmax_bits_x8(cur[u][2]), absmax_bits_x8(cur[u][3])));
+      ab = max_u16x2(ab, __shfl_xor_sync(FULL_MASK, ab, 1));
+      ab = max_u16x2(ab, __shfl_xor_sync(FULL_MASK, ab, 2));
+      const QScale qs = make_qscale(bits_to_absmax(ab));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint2 c = quant_bf16x8(cur[u][i], qs, ok);
+        if (ok) *reinterpret_cast<uint2*>(qr + (st0 + u) * 1024 + i * 32) = c;
       }
+      if (ok && sub == 0) sx[(int64_t)kb * ld_sx + m] = qs.s;
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) cur[u][i] = nxt[u][i];
   }
 }
 
 // ----------------------------------------------------------------------------------------------
 // a2: per-token (per-row) quantization.
 // Rows of at most 256 * CH elements: warp per row, the row in registers, shuffle reduction; each
-// warp walks rows m, m + nwarps, ... and loads its next row while it quantizes the current one.
+// warp walks rows m, m + nwarps, ...  PREFETCH: the next row is loaded while the current one is
+// quantized (used when warps own several rows); otherwise fewer registers give more resident
+// warps, so that one launch has every row in flight at once.
 // ----------------------------------------------------------------------------------------------
-template <int CH>
+template <int CH, bool PREFETCH>
 __global__ void __launch_bounds__(256) k_quant_act_token_warp(const uint16_t* __restrict__ x, int M, int K,
                                                               int64_t ldx, int8_t* __restrict__ xq,
                                                               float* __restrict__ sx) {
@@ -168,7 +205,7 @@ __global__ void __launch_bounds__(256) k_quant_act_token_warp(const uint16_t* __
   const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
   const int nv = K / 8;
-  uint4 cur[CH], nxt[CH];
+  uint4 cur[CH], nxt[PREFETCH ? CH : 1];
   auto load_row = [&](int m, uint4 (&v)[CH]) {
     const uint16_t* xr = x + (int64_t)m * ldx;
 #pragma unroll
@@ -181,7 +218,7 @@ __global__ void __launch_bounds__(256) k_quant_act_token_warp(const uint16_t* __
   int m = warp;
   if (m < M) load_row(m, cur);
   for (; m < M; m += nwarps) {
-    load_row(m + nwarps, nxt);
+    if constexpr (PREFETCH) load_row(m + nwarps, nxt);
     float a = 0.f;
 #pragma unroll
     for (int j = 0; j < CH; ++j) a = fmaxf(a, absmax_bf16x8(cur[j]));
@@ -197,8 +234,12 @@ __global__ void __launch_bounds__(256) k_quant_act_token_warp(const uint16_t* __
       if (ok) *reinterpret_cast<uint2*>(qr + c * 8) = code;
     }
     if (lane == 0) sx[m] = qs.s;
+    if constexpr (PREFETCH) {
 #pragma unroll
-    for (int j = 0; j < CH; ++j) cur[j] = nxt[j];
+      for (int j = 0; j < CH; ++j) cur[j] = nxt[j];
+    } else {
+      if (m + nwarps < M) load_row(m + nwarps, cur);
+    }
   }
 }
 

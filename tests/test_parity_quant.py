@@ -32,7 +32,7 @@ def _edge_activations(M, K, seed):
     return x
 
 
-@pytest.mark.parametrize("M,K", [(16, 512), (1, 128), (300, 1024), (37, 7168), (6, 18432)])
+@pytest.mark.parametrize("M,K", [(16, 512), (1, 128), (300, 1024), (37, 7168), (6, 18432), (9, 24576), (1000, 256)])
 def test_act_token_group(q, M, K):
     x = _edge_activations(M, K, seed=M + K)
     xq_ref, sx_ref = O.quant_act_token_group(x)
@@ -61,7 +61,7 @@ def test_act_token_group_strided_input(q):
     assert np.array_equal(host(sx)[:, :M].T, sx_ref)
 
 
-@pytest.mark.parametrize("M,K", [(16, 2048), (1, 16), (300, 2048), (6, 7168), (7, 18432), (130, 4096)])
+@pytest.mark.parametrize("M,K", [(16, 2048), (1, 16), (300, 2048), (6, 7168), (7, 18432), (130, 4096), (5, 24576), (1001, 384)])
 def test_act_token(q, M, K):
     x = _edge_activations(M, K, seed=2 * M + K)
     xq_ref, sx_ref = O.quant_act_token(x)
@@ -189,3 +189,53 @@ def test_quantizer_random_magnitudes(q):
     torch.cuda.synchronize()
     assert np.array_equal(host(xq), xq_ref)
     assert np.array_equal(host(sx).T, sx_ref)
+
+
+def _exhaustive_groups(exponents=(127, 100, 160)):
+    """Every absmax mantissa x every bf16 value below it (12 binades, both signs), as 128-groups.
+
+    The quantizer divides bf16 values v by s = RN(a / 127) with a bf16, so up to power-of-two
+    scaling this is its complete input domain (below 2^-11 a every code is 0)."""
+    rows = []
+    for ea in exponents:
+        for ma in range(128):
+            a_bits = (ea << 7) | ma
+            a = np.array([a_bits << 16], np.uint32).view(np.float32)[0]
+            ex = np.arange(ea - 11, ea + 1)
+            mant = np.arange(128)
+            bits = ((ex[:, None] << 7) | mant[None, :]).ravel().astype(np.uint32)
+            vals = (bits << 16).view(np.float32)
+            vals = vals[vals <= a]
+            vals = np.concatenate([vals, -vals])
+            for i in range(0, vals.size, 127):
+                row = np.zeros(128, np.float32)
+                row[0] = a
+                chunk = vals[i:i + 127]
+                row[1:1 + chunk.size] = chunk
+                rows.append(row)
+    return O.f32_to_bf16_rne(np.stack(rows))
+
+
+def test_quantizer_exhaustive_bf16_domain(q):
+    x = _exhaustive_groups()
+    M = x.shape[0]
+    xq_ref, sx_ref = O.quant_act_token_group(x)
+    xd = dev(x)
+    xq = empty((M, 128), torch.int8)
+    sx = empty((1, (M + 3) // 4 * 4), torch.float32)
+    q.i8q_quant_act_token_group(xd, xq, sx)
+    xq2 = empty((M, 128), torch.int8)
+    sx2 = empty((M,), torch.float32)
+    q.i8q_quant_act_token(xd, xq2, sx2)
+    # the same values as 128x128 weight blocks (rows padded to a multiple of 128)
+    Mp = (M + 127) // 128 * 128
+    xpad = np.zeros((Mp, 128), np.uint16)
+    xpad[:M] = x
+    wq = empty((Mp, 128), torch.int8)
+    sw = empty((Mp // 128, 1), torch.float32)
+    q.i8q_quant_weight_block(dev(xpad), wq, sw)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(xq), xq_ref) and np.array_equal(host(sx)[0, :M], sx_ref[:, 0])
+    assert np.array_equal(host(xq2), xq_ref) and np.array_equal(host(sx2), sx_ref[:, 0])
+    wq_ref, sw_ref = O.quant_weight_block(xpad)
+    assert np.array_equal(host(wq), wq_ref) and np.array_equal(host(sw), sw_ref)
