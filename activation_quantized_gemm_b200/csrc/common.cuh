@@ -184,6 +184,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 
 // Shared-memory matrix descriptor for a K-major operand stored with the 128-byte swizzle that
 // TMA (CU_TENSOR_MAP_SWIZZLE_128B) writes: rows of 128 bytes, 8-row core groups 1024 bytes

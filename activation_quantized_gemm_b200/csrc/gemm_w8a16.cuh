@@ -9,16 +9,18 @@
 //
 // Layout: "swap-AB" - the 128 weight rows of a tile are the MMA's M dimension, the (padded) tokens
 // its N dimension, so a decode batch of 1..64 tokens still fills the 128-row tensor-core tile.
-//   warp 0       TMA: int8 weight slab [128 rows x 128 K] (128B swizzle) + f16 activation slab
+//   warps 0..3   epilogue: thread = weight row; per slab, sum[m] += partial[m] * s[n][g].
+//   warps 4..7   converters: int8 slab (shared memory) -> exact f16 operand written straight into
+//                TMEM with tcgen05.st (NA operand buffers); the MMA reads its A operand from TMEM,
+//                so shared memory only carries the TMA-staged int8 weights and f16 activations.
+//   warp 8       TMA: int8 weight slab [128 rows x 128 K] (128B swizzle) + f16 activation slab
 //                [MP x 128 K] as two 64-element halves (128B swizzle), one mbarrier per stage.
-//   warp 1       TMEM allocation and MMA issue: 8 x tcgen05.mma.kind::f16 (K = 16) per slab.
-//   warps 4..11  converters: int8 slab -> f16 operand in shared memory (128B swizzle layout the
-//                MMA descriptor expects; NA operand buffers), then fence.proxy.async and an
-//                mbarrier arrival.
-//   warps 12..15 epilogue: thread = weight row; per slab, sum[m] += partial[m] * s[n][g].
-// Small-N MMAs have a long latency compared with their work, so consecutive MMAs never wait on
-// each other: each slab's 8 k-steps alternate between NACC independent TMEM accumulators (summed
-// by the epilogue), and up to NBUF slabs are in flight in a ring of TMEM accumulators.
+//   warp 9       TMEM allocation and MMA issue: 8 x tcgen05.mma.kind::f16 (K = 16) per slab.
+// For decode batches of up to 32 tokens two CTAs share an SM (256 TMEM columns each), so that a
+// single wave holds every CTA of the split-K grid.
+// Small-N MMAs have a long latency compared with their work, so consecutive MMAs do not wait on
+// each other: a slab's 8 k-steps are spread over NACC independent TMEM accumulators (each folded
+// into the running sum by the epilogue), and NBUF slabs are in flight in a ring of TMEM buffers.
 // Split-K: the CTAs of one thread-block cluster take disjoint slab ranges of the same 128 rows;
 // rank 0 adds the other ranks' fp32 partial tiles read from their shared memory (distributed
 // shared memory), in rank order, and writes fp16.
@@ -39,18 +41,20 @@ struct W8A16Cfg {
   static constexpr int X_HALF = MP * 128;               // one 64-element half of the f16 slab
   static constexpr int X_BYTES = 2 * X_HALF;
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
-  static constexpr int STAGES = MP >= 32 ? 4 : 6;
-  static constexpr int A_BYTES = W8A16_BN * 128 * 2;    // f16 operand of one slab: two 16 KB halves
-  static constexpr int NA = 3;                          // operand buffers
+  static constexpr int CTAS_PER_SM = MP <= 32 ? 2 : 1;  // two CTAs share an SM's TMEM and smem
+  static constexpr int STAGES = CTAS_PER_SM == 2 ? (MP <= 16 ? 5 : 4) : 6;
+  static constexpr int A_COLS = 64;                     // 128 K f16 values = 64 packed 32-bit columns
   static constexpr int NACC = 2;                        // independent accumulators per slab
-  static constexpr int NBUF = (512 / (NACC * MP)) < 8 ? (512 / (NACC * MP)) : 8;   // slab accumulators in TMEM
-  static constexpr int TMEM_NEED = NBUF * NACC * MP;
-  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
-                                   : TMEM_NEED <= 256 ? 256 : 512;
-  static constexpr int NUM_THREADS = 512;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NA * A_BYTES + 512 + 1024;
-  static_assert(MP * W8A16_BN * 4 <= NA * A_BYTES, "reduction tile must fit in the operand buffers");
-  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static constexpr int SLAB_COLS = NACC * MP;           // TMEM columns of one slab's partials
+  static constexpr int TMEM_COLS = CTAS_PER_SM == 2 ? 256 : 512;
+  static constexpr int NA = MP <= 16 ? 3 : 2;           // f16 operand buffers (in TMEM)
+  static constexpr int NBUF_FIT = (TMEM_COLS - NA * A_COLS) / SLAB_COLS;
+  static constexpr int NBUF = NBUF_FIT < 4 ? NBUF_FIT : 4;
+  static constexpr int NUM_THREADS = 320;               // warps 0-3 epilogue, 4-7 converters, 8 TMA, 9 MMA
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 512 + 1024;
+  static_assert(NBUF >= 2, "at least two slabs in flight");
+  static_assert(MP * W8A16_BN * 4 <= STAGES * STAGE_BYTES, "reduction tile must fit in the stage buffers");
+  static_assert(SMEM_BYTES * CTAS_PER_SM <= 232448, "shared memory");
 };
 
 struct W8A16Args {
@@ -79,8 +83,27 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
   return v;
 }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// D[tmem] (+)= A[tmem] * B[smem]^T, f16 x f16 -> f32 (K = 16); A is 128 lanes x 8 packed columns.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 registers -> 32 lanes x 32 columns of TMEM (thread t writes lane base + t)
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
 }
 
 // 4 signed int8 (one 32-bit word) -> 4 exact f16 values as two half2 words.
@@ -98,15 +121,14 @@ __device__ __forceinline__ void i8x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t
 }
 
 template <int MP>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
     k_gemm_w8a16(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const W8A16Args args) {
   using C = W8A16Cfg<MP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sStage = smem;                                   // STAGES x (W slab | X halves)
-  uint8_t* sA = smem + C::STAGES * C::STAGE_BYTES;          // NA x f16 operand (2 x 16 KB halves each)
-  uint64_t* full = reinterpret_cast<uint64_t*>(sA + C::NA * C::A_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* afull = empty + C::STAGES;
   uint64_t* aempty = afull + C::NA;
@@ -127,10 +149,10 @@ __global__ void __launch_bounds__(512, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 9);   // 8 converter warps + 1 MMA commit
+      mbar_init(&empty[s], 5);   // 4 converter warps + 1 MMA commit
     }
     for (int a = 0; a < C::NA; ++a) {
-      mbar_init(&afull[a], 8);
+      mbar_init(&afull[a], 4);
       mbar_init(&aempty[a], 1);
     }
     for (int b = 0; b < C::NBUF; ++b) {
@@ -141,11 +163,11 @@ __global__ void __launch_bounds__(512, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmX);
   }
-  if (warp == 1) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -158,7 +180,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
   for (int m = 0; m < MP; ++m) sum[m] = 0.f;
 
-  if (warp == 0) {
+  if (warp == 8) {
     if (lane == 0) {
       uint32_t filled = 0, fill_parity = 0;
       bool ok = true;
@@ -179,7 +201,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int s = 0; s < C::STAGES; ++s)
           if (filled & (1u << s)) mbar_wait(&full[s], (fill_parity >> s) & 1u, SITE_DRAIN, nullptr);
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(W8A16_BN, MP);
       for (int j = 0; j < nslab; ++j) {
@@ -193,14 +215,14 @@ __global__ void __launch_bounds__(512, 1)
         if (!mbar_wait(&afull[a], pa, SITE_CONVERT, abort_flag)) break;
         if (!mbar_wait(&full[s], ph, SITE_FULL, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + a * C::A_BYTES);
+        const uint32_t a0 = tmem + a * C::A_COLS;                       // operand columns
         const uint32_t x0 = smem_u32(sStage + s * C::STAGE_BYTES + C::W_BYTES);
-        const uint32_t d0 = tmem + b * C::NACC * MP;
+        const uint32_t d0 = tmem + C::NA * C::A_COLS + b * C::SLAB_COLS;  // accumulator columns
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t h = kk >> 2, off = (kk & 3) * 32;
-          mma_f16(d0 + (kk % C::NACC) * MP, sw128_kmajor_desc(a0 + h * 16384 + off),
-                  sw128_kmajor_desc(x0 + h * C::X_HALF + off), idesc, kk >= C::NACC);
+          mma_f16_ts(d0 + (kk % C::NACC) * MP, a0 + kk * 8, sw128_kmajor_desc(x0 + h * C::X_HALF + off), idesc,
+                     kk >= C::NACC);
         }
         tc_commit(&empty[s]);
         tc_commit(&aempty[a]);
@@ -209,12 +231,14 @@ __global__ void __launch_bounds__(512, 1)
       tc_commit(done);
       mbar_wait(done, 0, SITE_DRAIN, nullptr);
     }
-  } else if (warp >= 4 && warp < 12) {
-    // converters: warp c = warp - 4 owns weight rows 32 (c % 4) .. + 31 and K half c / 4 of the slab
-    const int c = warp - 4;
-    const int r = (c & 3) * 32 + lane;
-    const int h = c >> 2;
+  } else if (warp >= 4 && warp < 8) {
+    // converters: warp w owns weight rows 32 (w % 4) .. + 31 (its TMEM lane quarter); each thread
+    // writes the exact f16 values of its row's 128 K into the operand's TMEM columns (two f16 per
+    // 32-bit column, K order).
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
     const int sw = r & 7;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     for (int j = 0; j < nslab; ++j) {
       const int s = j % C::STAGES;
       const uint32_t ph = (j / C::STAGES) & 1;
@@ -222,30 +246,30 @@ __global__ void __launch_bounds__(512, 1)
       const uint32_t pa = (j / C::NA) & 1;
       if (!warp_wait(&full[s], ph, SITE_FULL, abort_flag)) break;
       if (!warp_wait(&aempty[a], pa ^ 1, SITE_CONVERT, abort_flag)) break;
+      tc_fence_after();
       const uint8_t* wrow = sStage + s * C::STAGE_BYTES + r * 128;
-      uint8_t* arow = sA + a * C::A_BYTES + h * 16384 + r * 128;
-      uint4 v[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(wrow + (((4 * h + i) ^ sw) << 4));
+      for (int h = 0; h < 2; ++h) {
+        uint32_t o[32];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint4 o0, o1;
-        i8x4_to_f16x4(v[i].x, o0.x, o0.y);
-        i8x4_to_f16x4(v[i].y, o0.z, o0.w);
-        i8x4_to_f16x4(v[i].z, o1.x, o1.y);
-        i8x4_to_f16x4(v[i].w, o1.z, o1.w);
-        // int8 chunk 4h + i holds f16 chunks 8h + 2i, 8h + 2i + 1: chunks 2i, 2i + 1 of operand half h
-        *reinterpret_cast<uint4*>(arow + (((2 * i) ^ sw) << 4)) = o0;
-        *reinterpret_cast<uint4*>(arow + (((2 * i + 1) ^ sw) << 4)) = o1;
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = *reinterpret_cast<const uint4*>(wrow + (((4 * h + i) ^ sw) << 4));
+          i8x4_to_f16x4(v.x, o[8 * i + 0], o[8 * i + 1]);
+          i8x4_to_f16x4(v.y, o[8 * i + 2], o[8 * i + 3]);
+          i8x4_to_f16x4(v.z, o[8 * i + 4], o[8 * i + 5]);
+          i8x4_to_f16x4(v.w, o[8 * i + 6], o[8 * i + 7]);
+        }
+        tmem_st32(tmem + lane_addr + a * C::A_COLS + h * 32, o);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&afull[a]);
         mbar_arrive(&empty[s]);
       }
     }
-  } else if (warp >= 12) {
+  } else if (warp < 4) {
     // epilogue: thread = weight row n0 + 32 * (warp % 4) + lane
     const int q = warp & 3;
     const int n = n0 + q * 32 + lane;
@@ -259,39 +283,39 @@ __global__ void __launch_bounds__(512, 1)
       if (j + 1 < nslab && n < N) sc_next = __half2float(__ushort_as_half(__ldg(args.s + (int64_t)n * G + kb0 + j + 1)));
       if (!warp_wait(&tfull[b], pb, SITE_TMEM_FULL, abort_flag)) break;
       tc_fence_after();
-      const uint32_t base = tmem + lane_addr + b * C::NACC * MP;
-      if constexpr (MP == 16) {
-        uint32_t p0[16], p1[16];
-        tmem_ld16(base, p0);
-        tmem_ld16(base + 16, p1);
+      const uint32_t base = tmem + lane_addr + C::NA * C::A_COLS + b * C::SLAB_COLS;
+      // every column c of the slab holds a partial of token c % MP: fold each into the running sum
+      if constexpr (C::SLAB_COLS == 32) {
+        uint32_t p0[32];
+        tmem_ld32(base, p0);
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[b]);
 #pragma unroll
-        for (int m = 0; m < 16; ++m) sum[m] = fmaf(__uint_as_float(p0[m]) + __uint_as_float(p1[m]), sc, sum[m]);
+        for (int j = 0; j < 32; ++j) sum[j % MP] = fmaf(__uint_as_float(p0[j]), sc, sum[j % MP]);
       } else {
+        static_assert(C::SLAB_COLS % 64 == 0, "slab columns");
 #pragma unroll
-        for (int c0 = 0; c0 < MP; c0 += 32) {
+        for (int c0 = 0; c0 < C::SLAB_COLS; c0 += 64) {
           uint32_t p0[32], p1[32];
           tmem_ld32(base + c0, p0);
-          tmem_ld32(base + MP + c0, p1);
+          tmem_ld32(base + c0 + 32, p1);
           tmem_ld_wait();
 #pragma unroll
-          for (int m = 0; m < 32; ++m) sum[c0 + m] = fmaf(__uint_as_float(p0[m]) + __uint_as_float(p1[m]), sc, sum[c0 + m]);
+          for (int j = 0; j < 32; ++j) sum[(c0 + j) % MP] = fmaf(__uint_as_float(p0[j]), sc, sum[(c0 + j) % MP]);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sum[(c0 + 32 + j) % MP] = fmaf(__uint_as_float(p1[j]), sc, sum[(c0 + 32 + j) % MP]);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[b]);
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[b]);
     }
   }
 
   // ---- split-K reduction across the cluster through distributed shared memory
-  float* red = reinterpret_cast<float*>(sA);   // [MP][128] fp32 partial tile (operand buffers are idle now)
+  float* red = reinterpret_cast<float*>(sStage);   // [MP][128] fp32 partial tile (the stages are idle now)
   tc_fence_before();
   __syncthreads();
-  const bool epi = warp >= 12;
+  const bool epi = warp < 4;
   const int row = epi ? (warp & 3) * 32 + lane : 0;
   if (epi && rank != 0) {
 #pragma unroll
@@ -312,7 +336,7 @@ __global__ void __launch_bounds__(512, 1)
   }
   cluster_sync_all();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace i8q

@@ -132,7 +132,6 @@ __device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
       "r"(v)
       : "memory");
 }
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_inc() {

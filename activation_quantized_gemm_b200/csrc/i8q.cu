@@ -207,7 +207,7 @@ static i8q_status launch_w8a16_mp(const uint16_t* x, const int8_t* wq, const uin
   st = make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, K, K, MP, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st) return st;
   const int64_t tiles = cdiv(N, W8A16_BN);
-  const int splits = w8a16_splits(tiles, K / 128, sms);
+  const int splits = w8a16_splits(tiles, K / 128, sms * C::CTAS_PER_SM);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits, 1);
   cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
