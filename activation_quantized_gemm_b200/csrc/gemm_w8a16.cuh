@@ -13,17 +13,18 @@
 //   warps 4..7   converters: int8 slab (shared memory) -> exact f16 operand written straight into
 //                TMEM with tcgen05.st (NA operand buffers); the MMA reads its A operand from TMEM,
 //                so shared memory only carries the TMA-staged int8 weights and f16 activations.
-//   warp 8       TMA: int8 weight slab [128 rows x 128 K] (128B swizzle) + f16 activation slab
-//                [MP x 128 K] as two 64-element halves (128B swizzle), one mbarrier per stage.
+//   warp 8       TMA: lane 0 fills the int8 weight ring ([128 rows x 128 K] slabs, 128B swizzle,
+//                released by the converters), lane 1 the f16 activation ring ([MP x 128 K] as two
+//                64-element halves, 128B swizzle, released by the MMA).
 //   warp 9       TMEM allocation and MMA issue: 8 x tcgen05.mma.kind::f16 (K = 16) per slab.
 // For decode batches of up to 32 tokens two CTAs share an SM (256 TMEM columns each), so that a
 // single wave holds every CTA of the split-K grid.
 // Small-N MMAs have a long latency compared with their work, so consecutive MMAs do not wait on
 // each other: a slab's 8 k-steps are spread over NACC independent TMEM accumulators (each folded
 // into the running sum by the epilogue), and NBUF slabs are in flight in a ring of TMEM buffers.
-// Split-K: the CTAs of one thread-block cluster take disjoint slab ranges of the same 128 rows;
-// rank 0 adds the other ranks' fp32 partial tiles read from their shared memory (distributed
-// shared memory), in rank order, and writes fp16.
+// Split-K: the CTAs of one thread-block cluster take disjoint slab ranges of the same 128 rows and
+// reduce-scatter their fp32 partial tiles through distributed shared memory (each CTA sums its
+// share of the rows over all ranks, in rank order, and writes fp16).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -40,9 +41,9 @@ struct W8A16Cfg {
   static constexpr int W_BYTES = W8A16_BN * 128;        // int8 slab
   static constexpr int X_HALF = MP * 128;               // one 64-element half of the f16 slab
   static constexpr int X_BYTES = 2 * X_HALF;
-  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
   static constexpr int CTAS_PER_SM = MP <= 32 ? 2 : 1;  // two CTAs share an SM's TMEM and smem
-  static constexpr int STAGES = CTAS_PER_SM == 2 ? (MP <= 16 ? 5 : 4) : 6;
+  static constexpr int W_STAGES = CTAS_PER_SM == 2 ? 5 : 8;   // weight ring (freed after conversion)
+  static constexpr int X_STAGES = MP <= 16 ? 4 : (MP <= 32 ? 3 : 4);   // activation ring (freed by the MMA)
   static constexpr int A_COLS = 64;                     // 128 K f16 values = 64 packed 32-bit columns
   static constexpr int NACC = 2;                        // independent accumulators per slab
   static constexpr int SLAB_COLS = NACC * MP;           // TMEM columns of one slab's partials
@@ -51,10 +52,12 @@ struct W8A16Cfg {
   static constexpr int NBUF_FIT = (TMEM_COLS - NA * A_COLS) / SLAB_COLS;
   static constexpr int NBUF = NBUF_FIT < 4 ? NBUF_FIT : 4;
   static constexpr int NUM_THREADS = 320;               // warps 0-3 epilogue, 4-7 converters, 8 TMA, 9 MMA
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 512 + 1024;
+  static constexpr int RING_BYTES = W_STAGES * W_BYTES + X_STAGES * X_BYTES;
+  static constexpr int SMEM_BYTES = RING_BYTES + 512 + 1024;
   static_assert(NBUF >= 2, "at least two slabs in flight");
-  static_assert(MP * W8A16_BN * 4 <= STAGES * STAGE_BYTES, "reduction tile must fit in the stage buffers");
-  static_assert(SMEM_BYTES * CTAS_PER_SM <= 232448, "shared memory");
+  static_assert(MP * W8A16_BN * 4 <= RING_BYTES, "reduction tile must fit in the ring buffers");
+  static_assert(MP % 4 == 0, "tokens are reduced four at a time");
+  static_assert(SMEM_BYTES * CTAS_PER_SM <= 229376, "shared memory");
 };
 
 struct W8A16Args {
@@ -76,11 +79,14 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
+// 16 bytes at the same shared-memory offset in CTA `rank` of the cluster (distributed shared memory)
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t local_addr, uint32_t rank) {
   uint32_t remote;
-  float v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  float4 v;
+  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(remote));
   return v;
 }
 // D[tmem] (+)= A[tmem] * B[smem]^T, f16 x f16 -> f32 (K = 16); A is 128 lanes x 8 packed columns.
@@ -127,10 +133,13 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
   using C = W8A16Cfg<MP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sStage = smem;                                   // STAGES x (W slab | X halves)
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* empty = full + C::STAGES;
-  uint64_t* afull = empty + C::STAGES;
+  uint8_t* sW = smem;                                       // W_STAGES x int8 weight slab
+  uint8_t* sX = smem + C::W_STAGES * C::W_BYTES;            // X_STAGES x f16 activation slab halves
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES);
+  uint64_t* wempty = wfull + C::W_STAGES;
+  uint64_t* xfull = wempty + C::W_STAGES;
+  uint64_t* xempty = xfull + C::X_STAGES;
+  uint64_t* afull = xempty + C::X_STAGES;
   uint64_t* aempty = afull + C::NA;
   uint64_t* tfull = aempty + C::NA;
   uint64_t* tempty = tfull + C::NBUF;
@@ -147,9 +156,13 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
   const int n0 = blockIdx.x * W8A16_BN;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 5);   // 4 converter warps + 1 MMA commit
+    for (int s = 0; s < C::W_STAGES; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 4);   // the 4 converter warps
+    }
+    for (int s = 0; s < C::X_STAGES; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);   // the MMA's commit
     }
     for (int a = 0; a < C::NA; ++a) {
       mbar_init(&afull[a], 4);
@@ -181,42 +194,52 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
   for (int m = 0; m < MP; ++m) sum[m] = 0.f;
 
   if (warp == 8) {
-    if (lane == 0) {
-      uint32_t filled = 0, fill_parity = 0;
+    // lane 0 feeds the weight ring (waits only for the converters), lane 1 the activation ring
+    // (waits only for the MMA); the two rings run ahead independently.
+    if (lane < 2) {
+      const bool is_w = lane == 0;
+      const int nst = is_w ? C::W_STAGES : C::X_STAGES;
+      uint64_t* fullb = is_w ? wfull : xfull;
+      uint64_t* emptyb = is_w ? wempty : xempty;
+      uint32_t filled = 0, par = 0;
       bool ok = true;
       for (int j = 0; j < nslab; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, SITE_EMPTY, abort_flag)) { ok = false; break; }
-        uint8_t* st = sStage + s * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+        const int st = j % nst;
+        const uint32_t ph = (j / nst) & 1;
         const int kk = (kb0 + j) * 128;
-        tma_load_2d(st, &tmW, &full[s], kk, n0);
-        tma_load_2d(st + C::W_BYTES, &tmX, &full[s], kk, 0);
-        tma_load_2d(st + C::W_BYTES + C::X_HALF, &tmX, &full[s], kk + 64, 0);
-        filled |= 1u << s;
-        fill_parity = (fill_parity & ~(1u << s)) | (ph << s);
+        if (!mbar_wait(&emptyb[st], ph ^ 1, SITE_EMPTY, abort_flag)) { ok = false; break; }
+        if (is_w) {
+          mbar_arrive_expect_tx(&fullb[st], C::W_BYTES);
+          tma_load_2d(sW + st * C::W_BYTES, &tmW, &fullb[st], kk, n0);
+        } else {
+          uint8_t* xs = sX + st * C::X_BYTES;
+          mbar_arrive_expect_tx(&fullb[st], C::X_BYTES);
+          tma_load_2d(xs, &tmX, &fullb[st], kk, 0);
+          tma_load_2d(xs + C::X_HALF, &tmX, &fullb[st], kk + 64, 0);
+        }
+        filled |= 1u << st;
+        par = (par & ~(1u << st)) | (ph << st);
       }
       if (!ok)
-        for (int s = 0; s < C::STAGES; ++s)
-          if (filled & (1u << s)) mbar_wait(&full[s], (fill_parity >> s) & 1u, SITE_DRAIN, nullptr);
+        for (int st = 0; st < nst; ++st)
+          if (filled & (1u << st)) mbar_wait(&fullb[st], (par >> st) & 1u, SITE_DRAIN, nullptr);
     }
   } else if (warp == 9) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(W8A16_BN, MP);
       for (int j = 0; j < nslab; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = (j / C::STAGES) & 1;
+        const int sx_ = j % C::X_STAGES;
+        const uint32_t px = (j / C::X_STAGES) & 1;
         const int a = j % C::NA;
         const uint32_t pa = (j / C::NA) & 1;
         const int b = j % C::NBUF;
         const uint32_t pb = (j / C::NBUF) & 1;
         if (!mbar_wait(&tempty[b], pb ^ 1, SITE_TMEM_EMPTY, abort_flag)) break;
         if (!mbar_wait(&afull[a], pa, SITE_CONVERT, abort_flag)) break;
-        if (!mbar_wait(&full[s], ph, SITE_FULL, abort_flag)) break;
+        if (!mbar_wait(&xfull[sx_], px, SITE_FULL, abort_flag)) break;
         tc_fence_after();
         const uint32_t a0 = tmem + a * C::A_COLS;                       // operand columns
-        const uint32_t x0 = smem_u32(sStage + s * C::STAGE_BYTES + C::W_BYTES);
+        const uint32_t x0 = smem_u32(sX + sx_ * C::X_BYTES);
         const uint32_t d0 = tmem + C::NA * C::A_COLS + b * C::SLAB_COLS;  // accumulator columns
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -224,7 +247,7 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
           mma_f16_ts(d0 + (kk % C::NACC) * MP, a0 + kk * 8, sw128_kmajor_desc(x0 + h * C::X_HALF + off), idesc,
                      kk >= C::NACC);
         }
-        tc_commit(&empty[s]);
+        tc_commit(&xempty[sx_]);
         tc_commit(&aempty[a]);
         tc_commit(&tfull[b]);
       }
@@ -240,14 +263,14 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
     const int sw = r & 7;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     for (int j = 0; j < nslab; ++j) {
-      const int s = j % C::STAGES;
-      const uint32_t ph = (j / C::STAGES) & 1;
+      const int sw_ = j % C::W_STAGES;
+      const uint32_t pw = (j / C::W_STAGES) & 1;
       const int a = j % C::NA;
       const uint32_t pa = (j / C::NA) & 1;
-      if (!warp_wait(&full[s], ph, SITE_FULL, abort_flag)) break;
+      if (!warp_wait(&wfull[sw_], pw, SITE_FULL, abort_flag)) break;
       if (!warp_wait(&aempty[a], pa ^ 1, SITE_CONVERT, abort_flag)) break;
       tc_fence_after();
-      const uint8_t* wrow = sStage + s * C::STAGE_BYTES + r * 128;
+      const uint8_t* wrow = sW + sw_ * C::W_BYTES + r * 128;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t o[32];
@@ -266,7 +289,7 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&afull[a]);
-        mbar_arrive(&empty[s]);
+        mbar_arrive(&wempty[sw_]);
       }
     }
   } else if (warp < 4) {
@@ -311,30 +334,56 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
     }
   }
 
-  // ---- split-K reduction across the cluster through distributed shared memory
-  float* red = reinterpret_cast<float*>(sStage);   // [MP][128] fp32 partial tile (the stages are idle now)
+  // ---- output.  Without a split the epilogue threads write their rows directly.  With a split,
+  // every CTA publishes its fp32 partial tile ([128 rows][MP] in shared memory) and CTA `rank` sums
+  // rows r with r % nrank == rank over all ranks, in rank order, 4 tokens per 16-byte load.
   tc_fence_before();
   __syncthreads();
-  const bool epi = warp < 4;
-  const int row = epi ? (warp & 3) * 32 + lane : 0;
-  if (epi && rank != 0) {
+  const int mlim = args.M < MP ? args.M : MP;
+  if (nrank == 1) {
+    if (warp < 4) {
+      const int n = n0 + warp * 32 + lane;
+      if (n < N) {
 #pragma unroll
-    for (int m = 0; m < MP; ++m) red[m * W8A16_BN + row] = sum[m];
-  }
-  cluster_sync_all();
-  if (epi && rank == 0) {
-    for (uint32_t r = 1; r < nrank; ++r) {
-#pragma unroll
-      for (int m = 0; m < MP; ++m) sum[m] += ld_dsmem_f32(smem_u32(&red[m * W8A16_BN + row]), r);
+        for (int m = 0; m < MP; ++m)
+          if (m < mlim) args.y[(int64_t)m * N + n] = __half_as_ushort(__float2half_rn(sum[m]));
+      }
     }
-    const int n = n0 + row;
-    if (n < N) {
+  } else {
+    float4* red = reinterpret_cast<float4*>(smem);   // [128][MP / 4] (the rings are idle now)
+    if (warp < 4) {
+      const int row = warp * 32 + lane;
 #pragma unroll
-      for (int m = 0; m < MP; ++m)
-        if (m < args.M) args.y[(int64_t)m * N + n] = __half_as_ushort(__float2half_rn(sum[m]));
+      for (int m4 = 0; m4 < MP / 4; ++m4)
+        red[row * (MP / 4) + m4] = make_float4(sum[4 * m4], sum[4 * m4 + 1], sum[4 * m4 + 2], sum[4 * m4 + 3]);
+    }
+    cluster_sync_all();
+    const int owned = (W8A16_BN - (int)rank + (int)nrank - 1) / (int)nrank;   // rows rank + i * nrank
+    const int items = owned * (MP / 4);
+    for (int e = threadIdx.x; e < items; e += C::NUM_THREADS) {
+      const int i = e / (MP / 4), m4 = e - (e / (MP / 4)) * (MP / 4);
+      const int row = (int)rank + i * (int)nrank;
+      const uint32_t la = smem_u32(&red[row * (MP / 4) + m4]);
+      float4 part[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p)
+        if (p < (int)nrank) part[p] = ld_dsmem_f32x4(la, (uint32_t)p);
+      float4 v = part[0];
+#pragma unroll
+      for (int p = 1; p < 8; ++p)
+        if (p < (int)nrank) {
+          v.x += part[p].x; v.y += part[p].y; v.z += part[p].z; v.w += part[p].w;
+        }
+      const int n = n0 + row;
+      if (n < N) {
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (4 * m4 + k < mlim) args.y[(int64_t)(4 * m4 + k) * N + n] = __half_as_ushort(__float2half_rn(vv[k]));
+      }
     }
   }
-  cluster_sync_all();
+  cluster_sync_all();   // no CTA leaves while its shared memory may still be read
   tc_fence_after();
   if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
 }

@@ -180,12 +180,15 @@ static int64_t resident_grid(Kern k, int threads, int sms) {
 }
 
 // ------------------------------------------------------------------ W8A16 launch ------------
-// Split-K factor: the cluster size s in 1..8 minimising (waves of CTAs) x (slabs per CTA).
-static int w8a16_splits(int64_t tiles, int64_t KB, int sms) {
+// Split-K factor: the cluster size s in 1..8 minimising (waves of CTAs) x (slabs per CTA), where a
+// wave is the CTA slots that clusters can occupy at once (about 95% of the SMs: cluster placement
+// within GPCs leaves a few SMs unused).
+static int w8a16_splits(int64_t tiles, int64_t KB, int sms, int per_sm) {
+  const int64_t slots = (int64_t)(sms * 95 / 100) * per_sm;
   int best = 1;
   int64_t best_cost = INT64_MAX;
   for (int s = 1; s <= 8 && s <= KB; ++s) {
-    const int64_t cost = cdiv(tiles * s, sms) * cdiv(KB, s);
+    const int64_t cost = cdiv(tiles * s, slots) * cdiv(KB, s);
     if (cost < best_cost) { best_cost = cost; best = s; }
   }
   return best;
@@ -207,7 +210,7 @@ static i8q_status launch_w8a16_mp(const uint16_t* x, const int8_t* wq, const uin
   st = make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, K, K, MP, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st) return st;
   const int64_t tiles = cdiv(N, W8A16_BN);
-  const int splits = w8a16_splits(tiles, K / 128, sms * C::CTAS_PER_SM);
+  const int splits = w8a16_splits(tiles, K / 128, sms, C::CTAS_PER_SM);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits, 1);
   cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
