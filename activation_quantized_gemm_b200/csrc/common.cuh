@@ -109,6 +109,22 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Pull a tile into L2 only (nothing reaches shared memory, no barrier).  L2 is the device's point
+// of coherence, so this is harmless even when the data is still being written by an earlier kernel:
+// such writes land in L2 and later loads see them.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y)
+               : "memory");
+}
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// start while the previous kernel on the stream is still running; grid_dependency_wait() blocks
+// until that kernel has completed and its memory is visible (it returns at once when there is no
+// such dependency).  grid_dependents_launch() lets the next kernel start early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -176,10 +176,12 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8 && lane == 0) {
-    prefetch_tmap(&tmW);
-    prefetch_tmap(&tmX);
-  }
+  // The kernel may be launched while the preceding kernel is still running: until
+  // grid_dependency_wait() it touches no global memory except L2 prefetches of its first weight
+  // slabs.  It lets the next kernel launch early in turn (that kernel waits for this one the same way).
+  grid_dependents_launch();
+  if (warp == 8 && lane == 0)
+    for (int j = 0; j < nslab && j < C::W_STAGES; ++j) tma_prefetch_l2_2d(&tmW, (kb0 + j) * 128, n0);
   if (warp == 9) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
@@ -188,6 +190,7 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();
 
   float sum[MP];
 #pragma unroll

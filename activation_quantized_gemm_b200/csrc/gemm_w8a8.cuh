@@ -218,9 +218,14 @@ __global__ void __launch_bounds__(384, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
+  // The kernel may be launched while the preceding kernel (typically the activation quantizer) is
+  // still running: until grid_dependency_wait() it touches no global memory except L2 prefetches of
+  // the weight slabs of its first tile.
+  if (warp == 0 && lane == 0 && pair < num_tiles) {
+    int mb, nb;
+    gemm_tile_coords(pair, Mt, Nt, mb, nb);
+    for (int kb = 0; kb < KB && kb < C::STAGES; ++kb)
+      tma_prefetch_l2_2d(&tmB, kb * GEMM_BK, nb * BN + (int)rank * HALF);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
@@ -230,6 +235,7 @@ __global__ void __launch_bounds__(384, 1)
   cluster_sync();   // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();
 
   if (warp < 4) {
     setmaxnreg_dec<24>();

@@ -1,0 +1,354 @@
+// Decode-size W8A8 GEMMs (M <= 64 tokens) for both schemes of "DeepSeek R1 INT8 quantization
+// practice on SGLang", section 2.3.  At these sizes the weights dominate the traffic, so the kernel
+// is built to stream them once from HBM:
+//
+// "Swap-AB" tcgen05.mma.kind::i8 (K = 32 per instruction): the 128 weight rows of a tile are the
+// MMA's M dimension, read by the tensor core straight from the TMA-staged 128B-swizzled shared
+// memory, and the (padded) tokens are its N dimension, so a batch of 1..64 tokens still fills the
+// 128-row tensor-core tile.  The thread-block cluster of a tile splits K; its CTAs reduce-scatter
+// their partial tiles through distributed shared memory (no global scratch).
+//   warps 0..3  epilogue: thread = weight row (TMEM lane).  Channel-wise: the exact int32 dot
+//               products are read once at the end, summed exactly over the cluster, then scaled by
+//               sx[m] * sw[n].  Block-wise: each 128-K slab has its own TMEM accumulator; its int32
+//               partial sums are folded into fp32 running sums with sx[m][kb] * sw[n/128][kb].
+//   warp 4      TMA producer: weight slab [128 rows x 128 K] + activation slab [MP x 128 K].
+//   warp 5      TMEM allocation and MMA issue (4 x tcgen05.mma per slab).
+// Two CTAs share an SM (rings of 4..6 stages each); the launch keeps all CTAs in one wave.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "gemm_w8a16.cuh"   // cluster helpers
+
+namespace i8q {
+
+constexpr int W8A8_SMALL_MAX_M = 64;
+
+// CPS CTAs share an SM; the stage ring fills the rest of its shared memory: under full streaming
+// load a weight slab takes about 2 us to arrive, so an SM needs of the order of 100 KB in flight.
+template <int MP, bool BLOCKWISE, int CPS>
+struct W8A8SmallCfg {
+  static constexpr int W_BYTES = 128 * 128;
+  static constexpr int X_BYTES = MP * 128;
+  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+  static constexpr int NBUF = BLOCKWISE ? 4 : 1;          // slab accumulators in TMEM
+  static constexpr int TMEM_NEED = NBUF * MP;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : 256;
+  static constexpr int NUM_THREADS = 192;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int RING_BYTES = 4 * 2 * MP * 4;      // block-wise scale-product rings, one per epilogue warp
+  static constexpr int FIXED_BYTES = BAR_BYTES + RING_BYTES + 1024;   // + 1024-byte alignment slack
+  static constexpr int SM_SMEM = 233472, CTA_RESERVED = 1024, CTA_MAX = 232448;
+  static constexpr int BUDGET = (SM_SMEM / CPS - CTA_RESERVED) < CTA_MAX ? (SM_SMEM / CPS - CTA_RESERVED) : CTA_MAX;
+  static constexpr int STAGES_FIT = (BUDGET - FIXED_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT < 16 ? STAGES_FIT : 16;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
+  static_assert(MP == 16 || MP == 32 || MP == 64, "MMA N");
+  static_assert(CPS == 1 || CPS == 2, "CTAs per SM");
+  static_assert(STAGES >= 4, "stage ring");
+  static_assert(MP * 128 * 4 <= STAGES * STAGE_BYTES, "reduction tile must fit in the stage buffers");
+  static_assert(CPS * (SMEM_BYTES + CTA_RESERVED) <= SM_SMEM && SMEM_BYTES <= CTA_MAX, "shared memory");
+};
+
+__device__ __forceinline__ int4 ld_dsmem_s32x4(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  int4 v;
+  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(remote));
+  return v;
+}
+
+// 32 lanes x CH columns of 32-bit TMEM (CH = 16 or 32)
+template <int CH>
+__device__ __forceinline__ void tmem_ld_ch(uint32_t taddr, uint32_t (&r)[CH]) {
+  if constexpr (CH == 16)
+    tmem_ld16(taddr, r);
+  else
+    tmem_ld32(taddr, r);
+}
+
+template <int MP, bool BLOCKWISE, int CPS, bool OUT_F32, bool DEBUG>
+__global__ void __launch_bounds__(192, CPS)
+    k_gemm_w8a8_small(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                      const W8A8Args args) {
+  using C = W8A8SmallCfg<MP, BLOCKWISE, CPS>;
+  constexpr int CH = MP < 32 ? MP : 32;   // TMEM columns per load
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + C::NBUF;
+  uint64_t* done = tempty + C::NBUF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = args.M, N = args.N, K = args.K;
+  const int KB = K / 128;
+  const uint32_t rank = cluster_ctarank(), nrank = cluster_nctarank();
+  const int kb0 = (int)((int64_t)KB * rank / nrank), kb1 = (int)((int64_t)KB * (rank + 1) / nrank);
+  const int nslab = kb1 - kb0;
+  const int n0 = blockIdx.x * 128;
+
+  // The kernel may be launched while the preceding kernel (typically the activation quantizer) is
+  // still running: until grid_dependency_wait() it touches no global memory except L2 prefetches of
+  // its first weight slabs, so that the weight stream starts as early as possible.  It lets the next
+  // kernel launch early in turn (that kernel waits for this one the same way).
+  grid_dependents_launch();
+  if (warp == 4 && lane == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < C::NBUF; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    for (int j = 0; j < nslab && j < C::STAGES; ++j) tma_prefetch_l2_2d(&tmW, (kb0 + j) * 128, n0);
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();
+
+  // per-thread results of the epilogue warps: channel: exact int32 dot products; block: fp32 sums
+  int32_t acc[MP];
+  float sum[MP];
+#pragma unroll
+  for (int m = 0; m < MP; ++m) {
+    acc[m] = 0;
+    sum[m] = 0.f;
+  }
+
+  if (warp == 4) {
+    if (lane == 0) {
+      uint32_t filled = 0, par = 0;
+      bool ok = true;
+      for (int j = 0; j < nslab; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t ph = (j / C::STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, SITE_EMPTY, abort_flag)) { ok = false; break; }
+        uint8_t* st = smem + s * C::STAGE_BYTES;
+        const int kk = (kb0 + j) * 128;
+        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+        tma_load_2d(st, &tmW, &full[s], kk, n0);
+        tma_load_2d(st + C::W_BYTES, &tmX, &full[s], kk, 0);
+        filled |= 1u << s;
+        par = (par & ~(1u << s)) | (ph << s);
+      }
+      if (!ok)
+        for (int s = 0; s < C::STAGES; ++s)
+          if (filled & (1u << s)) mbar_wait(&full[s], (par >> s) & 1u, SITE_DRAIN, nullptr);
+    }
+  } else if (warp == 5) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(128, MP);
+      for (int j = 0; j < nslab; ++j) {
+        const int s = j % C::STAGES;
+        const uint32_t ph = (j / C::STAGES) & 1;
+        const int b = BLOCKWISE ? j % C::NBUF : 0;
+        if (BLOCKWISE) {
+          if (!mbar_wait(&tempty[b], ((j / C::NBUF) & 1) ^ 1, SITE_TMEM_EMPTY, abort_flag)) break;
+        }
+        if (!mbar_wait(&full[s], ph, SITE_FULL, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t w0 = smem_u32(smem + s * C::STAGE_BYTES);
+        const uint32_t x0 = w0 + C::W_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint32_t accumulate = BLOCKWISE ? (uint32_t)(kk > 0) : (uint32_t)(j > 0 || kk > 0);
+          mma_i8(tmem + b * MP, sw128_kmajor_desc(w0 + kk * 32), sw128_kmajor_desc(x0 + kk * 32), idesc, accumulate);
+        }
+        tc_commit(&empty[s]);
+        if (BLOCKWISE) tc_commit(&tfull[b]);
+      }
+      if (!BLOCKWISE) tc_commit(&tfull[0]);
+      tc_commit(done);
+      mbar_wait(done, 0, SITE_DRAIN, nullptr);
+    }
+  } else {
+    // epilogue: thread = weight row n0 + 32 * warp + lane (TMEM lane quarter = warp)
+    const int row = warp * 32 + lane;
+    const int n = n0 + row;
+    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    if constexpr (!BLOCKWISE) {
+      if (nslab > 0 && warp_wait(&tfull[0], 0, SITE_TMEM_FULL, abort_flag)) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < MP / CH; ++c) {
+          uint32_t r[CH];
+          tmem_ld_ch<CH>(tmem + lane_addr + c * CH, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < CH; ++i) acc[c * CH + i] = (int32_t)r[i];
+        }
+      }
+    } else {
+      // Scale products sx[kb][m] * sw[tile][kb] of a slab go through a per-warp two-slot ring in
+      // shared memory: lane l loads token l (and l + 32) of slab j + 1 while slab j is folded, so
+      // the global-load latency is hidden behind one slab of streaming.
+      const float* swrow = args.sw + (int64_t)(n0 / 128) * KB;
+      float* ring = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES) + warp * 2 * MP;
+      constexpr int PER_LANE = (MP + 31) / 32;
+      float nsx[PER_LANE], nsw = 0.f;
+      auto load_scales = [&](int kb) {
+        nsw = __ldg(swrow + kb);
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) {
+          const int m = lane + 32 * i;
+          nsx[i] = (m < MP && m < M) ? __ldg(args.sx + (int64_t)kb * args.ld_sx + m) : 0.f;
+        }
+      };
+      if (nslab > 0) load_scales(kb0);
+      for (int j = 0; j < nslab; ++j) {
+        const int b = j % C::NBUF;
+        const int kb = kb0 + j;
+        float* slot = ring + (j & 1) * MP;
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i)
+          if (lane + 32 * i < MP) slot[lane + 32 * i] = nsx[i] * nsw;
+        __syncwarp();
+        if (j + 1 < nslab) load_scales(kb + 1);
+        if (!warp_wait(&tfull[b], (j / C::NBUF) & 1, SITE_TMEM_FULL, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < MP / CH; ++c) {
+          uint32_t r[CH];
+          tmem_ld_ch<CH>(tmem + lane_addr + b * MP + c * CH, r);
+          tmem_ld_wait();
+          if (c == MP / CH - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[b]);
+          }
+#pragma unroll
+          for (int i = 0; i < CH; i += 4) {
+            const float4 q = *reinterpret_cast<const float4*>(slot + c * CH + i);
+            sum[c * CH + i + 0] = fmaf(__int2float_rn((int)r[i + 0]), q.x, sum[c * CH + i + 0]);
+            sum[c * CH + i + 1] = fmaf(__int2float_rn((int)r[i + 1]), q.y, sum[c * CH + i + 1]);
+            sum[c * CH + i + 2] = fmaf(__int2float_rn((int)r[i + 2]), q.z, sum[c * CH + i + 2]);
+            sum[c * CH + i + 3] = fmaf(__int2float_rn((int)r[i + 3]), q.w, sum[c * CH + i + 3]);
+          }
+          if constexpr (DEBUG) {
+            if (n < N) {
+#pragma unroll
+              for (int i = 0; i < CH; ++i)
+                if (c * CH + i < M) args.dbg[((int64_t)(c * CH + i) * N + n) * KB + kb] = (int32_t)r[i];
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ---- output: reduce-scatter over the cluster (every CTA sums rows r % nrank == rank over all
+  // ranks, in rank order); without a split the epilogue threads write their rows directly.
+  tc_fence_before();
+  __syncthreads();
+  const int mlim = M < MP ? M : MP;
+  auto write_out = [&](int n, int m, float v) {
+    if (OUT_F32)
+      reinterpret_cast<float*>(args.y)[(int64_t)m * N + n] = v;
+    else
+      reinterpret_cast<uint16_t*>(args.y)[(int64_t)m * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  };
+  if (nrank == 1) {
+    if (warp < 4) {
+      const int n = n0 + warp * 32 + lane;
+      if (n < N) {
+        const float swn = BLOCKWISE ? 0.f : __ldg(args.sw + n);
+#pragma unroll
+        for (int m = 0; m < MP; ++m) {
+          if (m < mlim) {
+            if constexpr (BLOCKWISE) {
+              write_out(n, m, sum[m]);
+            } else {
+              write_out(n, m, __int2float_rn(acc[m]) * (__ldg(args.sx + m) * swn));
+              if constexpr (DEBUG) args.dbg[(int64_t)m * N + n] = acc[m];
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // partial tiles in [MP / 4][128 rows] of 4 x 32-bit (the stage buffers are idle now); CTA `rank`
+    // owns rows [128 * rank / nrank, 128 * (rank + 1) / nrank) and sums them over all ranks in rank order
+    uint4* red = reinterpret_cast<uint4*>(smem);
+    if (warp < 4) {
+      const int row = warp * 32 + lane;
+#pragma unroll
+      for (int m4 = 0; m4 < MP / 4; ++m4) {
+        if constexpr (BLOCKWISE)
+          red[m4 * 128 + row] = make_uint4(__float_as_uint(sum[4 * m4]), __float_as_uint(sum[4 * m4 + 1]),
+                                           __float_as_uint(sum[4 * m4 + 2]), __float_as_uint(sum[4 * m4 + 3]));
+        else
+          red[m4 * 128 + row] = make_uint4(acc[4 * m4], acc[4 * m4 + 1], acc[4 * m4 + 2], acc[4 * m4 + 3]);
+      }
+    }
+    cluster_sync_all();
+    const int r0 = (int)(128 * rank / nrank), r1 = (int)(128 * (rank + 1) / nrank);
+    const int owned = r1 - r0;
+    const int items = owned * ((mlim + 3) >> 2);
+    for (int e = threadIdx.x; e < items; e += C::NUM_THREADS) {
+      const int m4 = e / owned, row = r0 + (e - m4 * owned);
+      const int n = n0 + row;
+      const uint32_t la = smem_u32(&red[m4 * 128 + row]);
+      if constexpr (BLOCKWISE) {
+        float4 part[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+          if (p < (int)nrank) part[p] = ld_dsmem_f32x4(la, (uint32_t)p);
+        float4 v = part[0];
+#pragma unroll
+        for (int p = 1; p < 8; ++p)
+          if (p < (int)nrank) {
+            v.x += part[p].x; v.y += part[p].y; v.z += part[p].z; v.w += part[p].w;
+          }
+        if (n < N) {
+          const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (4 * m4 + k < mlim) write_out(n, 4 * m4 + k, vv[k]);
+        }
+      } else {
+        int4 part[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+          if (p < (int)nrank) part[p] = ld_dsmem_s32x4(la, (uint32_t)p);
+        int4 v = part[0];
+#pragma unroll
+        for (int p = 1; p < 8; ++p)
+          if (p < (int)nrank) {
+            v.x += part[p].x; v.y += part[p].y; v.z += part[p].z; v.w += part[p].w;
+          }
+        if (n < N) {
+          const int32_t vv[4] = {v.x, v.y, v.z, v.w};
+          const float swn = __ldg(args.sw + n);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int m = 4 * m4 + k;
+            if (m < mlim) {
+              write_out(n, m, __int2float_rn(vv[k]) * (__ldg(args.sx + m) * swn));
+              if constexpr (DEBUG) args.dbg[(int64_t)m * N + n] = vv[k];
+            }
+          }
+        }
+      }
+    }
+    cluster_sync_all();   // no CTA leaves while its shared memory may still be read
+  }
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace i8q

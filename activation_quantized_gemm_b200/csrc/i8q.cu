@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "gemm_w8a16.cuh"
 #include "gemm_w8a8.cuh"
+#include "gemm_w8a8_small.cuh"
 #include "quant.cuh"
 
 namespace i8q {
@@ -180,18 +181,26 @@ static int64_t resident_grid(Kern k, int threads, int sms) {
 }
 
 // ------------------------------------------------------------------ W8A16 launch ------------
-// Split-K factor: the cluster size s in 1..8 minimising (waves of CTAs) x (slabs per CTA), where a
-// wave is the CTA slots that clusters can occupy at once (about 95% of the SMs: cluster placement
-// within GPCs leaves a few SMs unused).
-static int w8a16_splits(int64_t tiles, int64_t KB, int sms, int per_sm) {
+// Split-K factor of the decode-size (weight-streaming) GEMMs: the smallest cluster size s in 1..8
+// that gives at least three quarters of the SMs a CTA (one CTA streams about 60 GB/s, so about 110
+// of them saturate HBM), without going past one wave of co-resident CTAs (about 95% of the SMs'
+// CTA slots: cluster placement within GPCs leaves a few SMs unused).  Every extra wave would pay
+// the per-CTA start-up and pipeline-fill latency again.
+static int decode_splits(int64_t tiles, int64_t KB, int sms, int per_sm) {
   const int64_t slots = (int64_t)(sms * 95 / 100) * per_sm;
-  int best = 1;
-  int64_t best_cost = INT64_MAX;
-  for (int s = 1; s <= 8 && s <= KB; ++s) {
-    const int64_t cost = cdiv(tiles * s, slots) * cdiv(KB, s);
-    if (cost < best_cost) { best_cost = cost; best = s; }
-  }
-  return best;
+  const int64_t target = (int64_t)sms * 3 / 4;
+  int s = 1;
+  while (s < 8 && s < KB && tiles * s < target && tiles * (s + 1) <= slots) ++s;
+  return s;
+}
+
+// Split-K factor of the decode-size W8A8 GEMM: the largest cluster size s in 1..8 (and <= K / 128)
+// whose tiles x s CTAs are all co-resident (CPS per SM), so that as many CTAs as fit stream weights
+// at once, in one wave.
+static int w8a8_small_splits(int64_t tiles, int64_t KB, int sms, int cps) {
+  int s = 1;
+  while (s < 8 && s < KB && tiles * (s + 1) <= (int64_t)sms * cps) ++s;
+  return s;
 }
 
 template <int MP>
@@ -210,19 +219,21 @@ static i8q_status launch_w8a16_mp(const uint16_t* x, const int8_t* wq, const uin
   st = make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, K, K, MP, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st) return st;
   const int64_t tiles = cdiv(N, W8A16_BN);
-  const int splits = w8a16_splits(tiles, K / 128, sms, C::CTAS_PER_SM);
+  const int splits = decode_splits(tiles, K / 128, sms, C::CTAS_PER_SM);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits, 1);
   cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 1;
   at[0].val.clusterDim.y = (unsigned)splits;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see grid_dependency_wait()
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   W8A16Args a{s, M, N, K, y};
   I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, tw, tx, a));
   return I8Q_OK;
@@ -272,16 +283,65 @@ static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args
   cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = s;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see grid_dependency_wait()
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, a));
   return I8Q_OK;
 }
+
+// Decode-size batches (M <= 64): weight rows on the MMA's M side, tokens padded to 16/32/64 on its
+// N side, K split over a thread-block cluster.
+template <int MP, bool BLOCKWISE, bool F32, bool DBG>
+static i8q_status launch_w8a8_small_mp(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms,
+                                       cudaStream_t s) {
+  constexpr int CPS = 2;
+  using C = W8A8SmallCfg<MP, BLOCKWISE, CPS>;
+  auto kern = k_gemm_w8a8_small<MP, BLOCKWISE, CPS, F32, DBG>;
+  static std::once_flag once;
+  static i8q_status attr = I8Q_OK;
+  std::call_once(once, [&] { attr = set_smem(kern, C::SMEM_BYTES); });
+  if (attr) return attr;
+  CUtensorMap tw, tx;
+  i8q_status st = make_tmap_2d(&tw, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, a.K, 128, 128,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  st = make_tmap_2d(&tx, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, a.K, MP, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  const int64_t tiles = cdiv(a.N, 128);
+  const int splits = w8a8_small_splits(tiles, a.K / 128, sms, CPS);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits, 1);
+  cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = (unsigned)splits;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see grid_dependency_wait()
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, tw, tx, a));
+  return I8Q_OK;
+}
+
+template <bool BLOCKWISE, bool F32, bool DBG>
+static i8q_status launch_w8a8_any(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms, cudaStream_t s) {
+  if (a.M <= 16) return launch_w8a8_small_mp<16, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
+  if (a.M <= 32) return launch_w8a8_small_mp<32, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
+  if (a.M <= W8A8_SMALL_MAX_M) return launch_w8a8_small_mp<64, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
+  return launch_w8a8<256, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
+}
+
 
 }  // namespace i8q
 
@@ -443,10 +503,9 @@ i8q_status i8q_gemm_w8a8_channel(const int8_t* xq, const float* sx, const int8_t
     if (dbg) I8Q_CUDA(cudaMemsetAsync(dbg, 0, (size_t)M * N * 4, S(stream)));
     return I8Q_OK;
   }
-  constexpr int BN = 256;
   W8A8Args a{sx, 0, sw, (int)M, (int)N, (int)K, y, dbg};
-  if (dbg) return launch_w8a8<BN, false, false, true>(xq, wq, a, sms, S(stream));
-  return launch_w8a8<BN, false, false, false>(xq, wq, a, sms, S(stream));
+  if (dbg) return launch_w8a8_any<false, false, true>(xq, wq, a, sms, S(stream));
+  return launch_w8a8_any<false, false, false>(xq, wq, a, sms, S(stream));
 }
 
 i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx, const int8_t* wq, const float* sw,
@@ -464,15 +523,14 @@ i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx,
     I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * osz, S(stream)));
     return I8Q_OK;
   }
-  constexpr int BN = 256;
   W8A8Args a{sx, ld_sx, sw, (int)M, (int)N, (int)K, y, dbg};
   const bool f32 = out == I8Q_OUT_FP32;
   if (dbg) {
-    if (f32) return launch_w8a8<BN, true, true, true>(xq, wq, a, sms, S(stream));
-    return launch_w8a8<BN, true, false, true>(xq, wq, a, sms, S(stream));
+    if (f32) return launch_w8a8_any<true, true, true>(xq, wq, a, sms, S(stream));
+    return launch_w8a8_any<true, false, true>(xq, wq, a, sms, S(stream));
   }
-  if (f32) return launch_w8a8<BN, true, true, false>(xq, wq, a, sms, S(stream));
-  return launch_w8a8<BN, true, false, false>(xq, wq, a, sms, S(stream));
+  if (f32) return launch_w8a8_any<true, true, false>(xq, wq, a, sms, S(stream));
+  return launch_w8a8_any<true, false, false>(xq, wq, a, sms, S(stream));
 }
 
 // ---------------------------------------------------------------- a6 -------------------------

@@ -15,7 +15,11 @@ from gpu_util import dev, empty, host, setup_library
 pytestmark = pytest.mark.gpu
 
 SHAPES = [(1, 8, 128), (16, 256, 512), (7, 200, 384), (130, 264, 1024), (300, 520, 2048),
-          (129, 1032, 768), (260, 136, 128)]
+          (129, 1032, 768), (260, 136, 128),
+          # decode-size batches (M <= 64): token padding to 16 / 32 / 64, K split over clusters of
+          # 1..8 CTAs with slab counts that do not divide evenly, ragged last weight tile
+          (17, 136, 896), (33, 520, 1152), (64, 1032, 4096), (48, 8, 256), (2, 2056, 1920),
+          (65, 264, 1024)]
 
 
 @pytest.fixture(scope="module")
