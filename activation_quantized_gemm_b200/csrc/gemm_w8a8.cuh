@@ -49,9 +49,10 @@ struct W8A8Cfg {
   static constexpr int NUM_THREADS = 384;
   static constexpr int EPI_WARPS = 8;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr int EPI_STAGE_BYTES = EPI_WARPS * 32 * 80;   // per epilogue warp: 32 rows x 80 B
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + EPI_STAGE_BYTES + 1024;  // + alignment slack
   static_assert(2 * BN <= TMEM_COLS, "two accumulators must fit in TMEM");
-  static_assert(BN % 32 == 0 && BN <= 256, "MMA N");
+  static_assert(BN % 32 == 0 && BN <= 256, "MMA N (each CTA's BN / 2 weight rows: whole 8-row groups)");
 };
 
 struct W8A8Args {
@@ -178,6 +179,33 @@ __device__ __forceinline__ void store_row8(void* y, bool f32out, int64_t off, co
   }
 }
 
+// One warp's row-per-thread bf16 results -> global memory with whole-sector stores: lane l holds
+// columns nc .. nc + W - 1 (W = 16 or 32) of row m_base + l as bf16 pairs.  The 32 rows go through
+// a 32 x 80-byte staging slab in shared memory (80-byte rows: conflict-free for row-wise writes and
+// column-wise reads), then each store instruction writes 8 rows x 64 contiguous bytes instead of
+// 16 bytes of 32 different rows (half-filled sectors).
+__device__ __forceinline__ void store_rows_bf16(uint8_t* stg, int lane, const uint32_t (&p)[16], int W, uint16_t* y,
+                                                int N, int m_base, int M, int nc) {
+  uint4* srow = reinterpret_cast<uint4*>(stg + lane * 80);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (q * 8 < W) srow[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = i * 8 + (lane & 7), c = lane >> 3;
+    const int m = m_base + r, n = nc + c * 8;
+    if (c * 8 < W && m < M && n < N)
+      *reinterpret_cast<uint4*>(y + (int64_t)m * N + n) = *reinterpret_cast<const uint4*>(stg + r * 80 + c * 16);
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 template <int BN, bool BLOCKWISE, bool OUT_F32, bool DEBUG>
 __global__ void __launch_bounds__(384, 1)
     k_gemm_w8a8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -196,6 +224,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* sStage = smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cta_rank_in_cluster();
@@ -321,6 +350,7 @@ __global__ void __launch_bounds__(384, 1)
     const int h = (warp - 4) >> 2;                  // column half
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     const int row = (int)rank * 128 + q * 32 + lane;  // row within the 256-row pair tile
+    uint8_t* stg = sStage + (warp - 4) * 32 * 80;     // this warp's store staging slab
     const uint32_t tempty_leader0 = map_to_rank(&tempty[0], 0), tempty_leader1 = map_to_rank(&tempty[1], 0);
     uint32_t acc_iter = 0;
 
@@ -350,25 +380,26 @@ __global__ void __launch_bounds__(384, 1)
         if (!warp_wait(&tfull[acc], (acc_iter >> 1) & 1, SITE_TMEM_FULL, abort_flag)) break;
         tc_fence_after();
         const float sxm = row_ok ? __ldg(args.sx + m) : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < HALF / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_addr + acc * BN + h * HALF + c * 32, r);
-          tmem_ld_wait();
-          const int nc = n0 + c * 32;
-          if (row_ok) {
+        // scale W columns starting at column nc of the row and store them (whole-sector stores)
+        auto emit = [&](const uint32_t* r, int nc, int W) {
+          uint32_t pk[16];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              const int n = nc + g * 8;
+          for (int g = 0; g < 4; ++g) {
+            const int n = nc + g * 8;
+            if (g * 8 < W) {
+              float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
               if (n < N) {
-                const float4 w0 = __ldg(reinterpret_cast<const float4*>(args.sw + n));
-                const float4 w1 = __ldg(reinterpret_cast<const float4*>(args.sw + n + 4));
-                const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                float v[8];
+                w0 = __ldg(reinterpret_cast<const float4*>(args.sw + n));
+                w1 = __ldg(reinterpret_cast<const float4*>(args.sw + n + 4));
+              }
+              const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+              float v[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = __int2float_rn((int)r[g * 8 + j]) * (sxm * ws[j]);
-                store_row8(args.y, false, (int64_t)m * N + n, v);
-                if constexpr (DEBUG) {
+              for (int j = 0; j < 8; ++j) v[j] = __int2float_rn((int)r[g * 8 + j]) * (sxm * ws[j]);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) pk[g * 4 + j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+              if constexpr (DEBUG) {
+                if (row_ok && n < N) {
                   int4* dp = reinterpret_cast<int4*>(args.dbg + (int64_t)m * N + n);
                   dp[0] = make_int4(r[g * 8 + 0], r[g * 8 + 1], r[g * 8 + 2], r[g * 8 + 3]);
                   dp[1] = make_int4(r[g * 8 + 4], r[g * 8 + 5], r[g * 8 + 6], r[g * 8 + 7]);
@@ -376,6 +407,21 @@ __global__ void __launch_bounds__(384, 1)
               }
             }
           }
+          store_rows_bf16(stg, lane, pk, W, reinterpret_cast<uint16_t*>(args.y), N, m - lane, M, nc);
+        };
+#pragma unroll 1
+        for (int c = 0; c < HALF / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_addr + acc * BN + h * HALF + c * 32, r);
+          tmem_ld_wait();
+          emit(r, n0 + c * 32, 32);
+        }
+        if constexpr (HALF % 32 == 16) {   // 16-column tail of a 224- or 160-column tile
+          uint32_t r[32];
+          tmem_ld16(tmem + lane_addr + acc * BN + h * HALF + (HALF / 32) * 32,
+                    *reinterpret_cast<uint32_t(*)[16]>(r));
+          tmem_ld_wait();
+          emit(r, n0 + (HALF / 32) * 32, 16);
         }
         tc_fence_before();
         __syncwarp();
@@ -434,19 +480,29 @@ __global__ void __launch_bounds__(384, 1)
           ++acc_iter;
         }
         if (!ok) break;
-        if (live) {
+        if constexpr (OUT_F32) {   // 8 fp32 = 32 bytes: whole sectors already
+          if (live) {
 #pragma unroll
-          for (int g = 0; g < HALF / 8; ++g) {
-            const int n = n0 + g * 8;
-            if (n < N) {
-              float v[8];
+            for (int g = 0; g < HALF / 8; ++g) {
+              const int n = n0 + g * 8;
+              if (n < N) {
+                float v[8];
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                v[2 * j] = sum[g * 4 + j].x;
-                v[2 * j + 1] = sum[g * 4 + j].y;
+                for (int j = 0; j < 4; ++j) {
+                  v[2 * j] = sum[g * 4 + j].x;
+                  v[2 * j + 1] = sum[g * 4 + j].y;
+                }
+                store_row8(args.y, true, (int64_t)m * N + n, v);
               }
-              store_row8(args.y, OUT_F32, (int64_t)m * N + n, v);
             }
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < HALF / 32; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(sum[c * 16 + j].x, sum[c * 16 + j].y);
+            store_rows_bf16(stg, lane, pk, 32, reinterpret_cast<uint16_t*>(args.y), N, m - lane, M, n0 + c * 32);
           }
         }
       }

@@ -334,11 +334,35 @@ static i8q_status launch_w8a8_small_mp(const int8_t* xq, const int8_t* wq, const
   return I8Q_OK;
 }
 
+// Tile width of the channel-wise pair tiles (256 x BN): the persistent pairs run ceil(tiles / pairs)
+// rounds of work proportional to BN (+ a fixed cost per tile), so a narrower tile wins when it
+// fills the last round better (M = 4096, N = 7168: 448 tiles of 256 leave 70 of 74 pairs idle in
+// the 7th round; 512 tiles of 224 fill it).
+static int channel_tile_n(int64_t M, int64_t N, int sms) {
+  const int64_t pairs = sms / 2;
+  const int cands[3] = {256, 224, 192};
+  int best = 256;
+  int64_t best_cost = INT64_MAX;
+  for (int bn : cands) {
+    const int64_t tiles = cdiv(M, GEMM_BM) * cdiv(N, bn);
+    const int64_t cost = cdiv(tiles, pairs) * (bn + 32);
+    if (cost < best_cost) { best_cost = cost; best = bn; }
+  }
+  return best;
+}
+
 template <bool BLOCKWISE, bool F32, bool DBG>
 static i8q_status launch_w8a8_any(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms, cudaStream_t s) {
   if (a.M <= 16) return launch_w8a8_small_mp<16, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
   if (a.M <= 32) return launch_w8a8_small_mp<32, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
   if (a.M <= W8A8_SMALL_MAX_M) return launch_w8a8_small_mp<64, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
+  if constexpr (!BLOCKWISE) {
+    switch (channel_tile_n(a.M, a.N, sms)) {
+      case 224: return launch_w8a8<224, false, F32, DBG>(xq, wq, a, sms, s);
+      case 192: return launch_w8a8<192, false, F32, DBG>(xq, wq, a, sms, s);
+      default: break;
+    }
+  }
   return launch_w8a8<256, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
 }
 
