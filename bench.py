@@ -10,11 +10,13 @@ the offline requantization and the W8A16 decode GEMM.
 
 Timing: W warm-up steps, then K steps back to back between CUDA events on the launching stream,
 cycling through enough independent copies of every input and output that the working set of a
-cycle exceeds twice the 126 MB L2 (no step reads what the previous one left in L2).  Each
-kernel of a step is bracketed by its own events, so the dominant kernel's average duration is
-measured live.  With torchrun (N > 1) every rank runs the same per-GPU workload on its own
-tokens (data-parallel, weights replicated, no collective on the data path): weak scaling,
-value = all ranks' work / max-over-ranks time.
+cycle exceeds twice the 126 MB L2 (no step reads what the previous one left in L2).  The timed
+region holds only the steps' kernels, so a GEMM may overlap its start-up with the kernel before
+it (programmatic dependent launch).  A second pass of K steps brackets every kernel with its own
+events, which gives each kernel's average launch duration (the roofline figure).  With torchrun
+(N > 1) every rank runs the same per-GPU workload on its own tokens (data-parallel, weights
+replicated, no collective on the data path): weak scaling, value = all ranks' work /
+max-over-ranks time.
 
 `--impl reference` times the CPU oracle (tests' reference implementation) on a bounded sample
 of the same workload instead.
@@ -49,6 +51,30 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+# ------------------------------------------------------------------- data-parallel host logic
+
+def shard_seed(base: int, rank: int) -> int:
+    """Seed of a rank's activations: every rank draws its own tokens; weights use `base` alone
+    (replicated)."""
+    return base + 1000 * rank
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The largest of every rank's value (a job ends when its slowest rank does)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_step: float, steps: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the work of every rank's steps over the max-over-ranks time."""
+    return units_per_step * steps * world / (ms / 1e3)
+
+
 # ---------------------------------------------------------------------------------- workloads
 
 class Workload:
@@ -78,7 +104,7 @@ class ChannelW8A8(Workload):
         self.q = i8q
         M, N, K = args.M or 4096, 7168, 2048
         self.M, self.N, self.K = M, N, K
-        x = synth.activation_bf16(M, K, seed=1 + 1000 * rank, outlier_p=0.001, outlier_mult=50.0)
+        x = synth.activation_bf16(M, K, seed=shard_seed(1, rank), outlier_p=0.001, outlier_mult=50.0)
         w = synth.weight_bf16(N, K, seed=1)
         self.x_host = torch.from_numpy(x.view(np.int16)).pin_memory()
         per_copy = M * K * 3 + 4 * M + N * K + 4 * N + 2 * M * N
@@ -158,7 +184,7 @@ class BlockW8A8(Workload):
         N, K = (18432, 7168) if proj == "up" else (7168, 18432)
         M = args.M or 4096
         self.M, self.N, self.K = M, N, K
-        x = synth.activation_bf16(M, K, seed=2 + 1000 * rank, outlier_p=0.001, outlier_mult=50.0)
+        x = synth.activation_bf16(M, K, seed=shard_seed(2, rank), outlier_p=0.001, outlier_mult=50.0)
         w = synth.weight_bf16(N, K, seed=2)
         self.x_host = torch.from_numpy(x.view(np.int16)).pin_memory()
         KB = K // 128
@@ -290,7 +316,7 @@ class W8A16(Workload):
         M = args.M or 16
         N, K = (12288, 4096) if args.proj == "up" else (4096, 12288)
         self.M, self.N, self.K = M, N, K
-        x = synth.activation_f16(M, K, seed=4 + 1000 * rank)
+        x = synth.activation_f16(M, K, seed=shard_seed(4, rank))
         wq, s = synth.int8_weight_groups(N, K, seed=4)
         per_copy = N * K + 2 * N * (K // 128) + 2 * M * K + 2 * M * N
         self.R = _rotations(per_copy)
@@ -452,10 +478,7 @@ def run_ours(args):
     total_ms = t_start.elapsed_time(t_end)
     per_kernel_ms = [sum(ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(args.steps)) / args.steps
                      for k in range(nk)]
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, "cuda")
 
     # end to end through the public API: pinned host input -> device, step, result -> host
     for i in range(2):
@@ -470,10 +493,7 @@ def run_ours(args):
     e1.record(stream)
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, "cuda")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -494,8 +514,8 @@ def run_ours(args):
             achieved = wl.dom_bytes / 1e9 / (dom_ms / 1e3)
             unit = "GB/s"
             peak_note = f"{src} HBM copy bandwidth"
-        value = wl.units_per_step * args.steps * world / (total_ms / 1e3)
-        e2e_value = wl.units_per_step * args.steps * world / (e2e_ms / 1e3)
+        value = job_throughput(wl.units_per_step, args.steps, world, total_ms)
+        e2e_value = job_throughput(wl.units_per_step, args.steps, world, e2e_ms)
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": wl.unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
