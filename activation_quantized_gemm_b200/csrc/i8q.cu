@@ -180,6 +180,24 @@ static int64_t resident_grid(Kern k, int threads, int sms) {
   return (int64_t)per_sm * sms;
 }
 
+// Launch with programmatic stream serialization (the kernel calls grid_dependency_wait() before
+// its first global-memory access).
+template <typename... KArgs, typename... Args>
+static i8q_status launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
+  return I8Q_OK;
+}
+
 // ------------------------------------------------------------------ W8A16 launch ------------
 // Split-K factor of the decode-size (weight-streaming) GEMMs: the smallest cluster size s in 1..8
 // that gives at least three quarters of the SMs a CTA (one CTA streams about 60 GB/s, so about 110
@@ -424,7 +442,8 @@ i8q_status i8q_quant_act_token_group(const uint16_t* x, int64_t M, int64_t K, in
   int64_t blocks = cdiv(items, 8);
   const int64_t cap = resident_grid(k_quant_act_token_group<U>, 256, sms);
   if (blocks > cap) blocks = cap;
-  k_quant_act_token_group<U><<<(unsigned)blocks, 256, 0, S(stream)>>>(x, (int)M, (int)KB, ldx, xq, sx, ld_sx);
+  st = launch_pdl(k_quant_act_token_group<U>, (unsigned)blocks, 256, S(stream), x, (int)M, (int)KB, ldx, xq, sx, ld_sx);
+  if (st) return st;
   I8Q_LAUNCHED("k_quant_act_token_group");
   return I8Q_OK;
 }
@@ -448,20 +467,21 @@ i8q_status i8q_quant_act_token(const uint16_t* x, int64_t M, int64_t K, int64_t 
     if (cdiv(warps, 8) <= cap1) {          // every row in flight at once: no prefetch needed
       const unsigned grid = (unsigned)cdiv(warps, 8);
       if (nv <= 32 * 2)
-        k_quant_act_token_warp<2, false><<<grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+        st = launch_pdl(k_quant_act_token_warp<2, false>, grid, 256, S(stream), x, (int)M, (int)K, ldx, xq, sx);
       else if (nv <= 32 * 4)
-        k_quant_act_token_warp<4, false><<<grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+        st = launch_pdl(k_quant_act_token_warp<4, false>, grid, 256, S(stream), x, (int)M, (int)K, ldx, xq, sx);
       else
-        k_quant_act_token_warp<8, false><<<grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+        st = launch_pdl(k_quant_act_token_warp<8, false>, grid, 256, S(stream), x, (int)M, (int)K, ldx, xq, sx);
     } else {                                 // warps own several rows: prefetch the next
       int64_t grid = cdiv(M, 8);
       const int64_t cap = resident_grid(k_quant_act_token_warp<8, true>, 256, sms);
       if (grid > cap) grid = cap;
-      k_quant_act_token_warp<8, true><<<(unsigned)grid, 256, 0, S(stream)>>>(x, (int)M, (int)K, ldx, xq, sx);
+      st = launch_pdl(k_quant_act_token_warp<8, true>, (unsigned)grid, 256, S(stream), x, (int)M, (int)K, ldx, xq, sx);
     }
   } else {              // CTA per row
-    k_quant_act_token_cta<<<(unsigned)M, 256, 0, S(stream)>>>(x, (int)K, ldx, xq, sx);
+    st = launch_pdl(k_quant_act_token_cta, (unsigned)M, 256, S(stream), x, (int)K, ldx, xq, sx);
   }
+  if (st) return st;
   I8Q_LAUNCHED("k_quant_act_token");
   return I8Q_OK;
 }

@@ -133,7 +133,12 @@ template <int U>
 __global__ void __launch_bounds__(256) k_quant_act_token_group(const uint16_t* __restrict__ x, int M, int KB,
                                                                int64_t ldx, int8_t* __restrict__ xq,
                                                                float* __restrict__ sx, int64_t ld_sx) {
-  grid_dependents_launch();   // a GEMM launched behind this kernel may start its prologue now
+  // Launched with programmatic stream serialization: the launch may overlap the end of the kernel
+  // before it (often the GEMM that produced x, or one that still reads the xq / sx being
+  // overwritten), so no global memory is touched before that kernel has completed.  A GEMM
+  // launched behind this kernel may start its prologue at once.
+  grid_dependents_launch();
+  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int gl = lane >> 2;                        // group within the warp step (0..7)
   const int sub = lane & 3;                        // lane within the group
@@ -202,7 +207,12 @@ template <int CH, bool PREFETCH>
 __global__ void __launch_bounds__(256) k_quant_act_token_warp(const uint16_t* __restrict__ x, int M, int K,
                                                               int64_t ldx, int8_t* __restrict__ xq,
                                                               float* __restrict__ sx) {
-  grid_dependents_launch();   // a GEMM launched behind this kernel may start its prologue now
+  // Launched with programmatic stream serialization: the launch may overlap the end of the kernel
+  // before it (often the GEMM that produced x, or one that still reads the xq / sx being
+  // overwritten), so no global memory is touched before that kernel has completed.  A GEMM
+  // launched behind this kernel may start its prologue at once.
+  grid_dependents_launch();
+  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int warp = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int nwarps = (int)((gridDim.x * blockDim.x) >> 5);
@@ -258,7 +268,12 @@ __device__ __forceinline__ float block_absmax(float a, float* red, int nwarps) {
 
 __global__ void __launch_bounds__(256) k_quant_act_token_cta(const uint16_t* __restrict__ x, int K, int64_t ldx,
                                                              int8_t* __restrict__ xq, float* __restrict__ sx) {
-  grid_dependents_launch();   // a GEMM launched behind this kernel may start its prologue now
+  // Launched with programmatic stream serialization: the launch may overlap the end of the kernel
+  // before it (often the GEMM that produced x, or one that still reads the xq / sx being
+  // overwritten), so no global memory is touched before that kernel has completed.  A GEMM
+  // launched behind this kernel may start its prologue at once.
+  grid_dependents_launch();
+  grid_dependency_wait();
   __shared__ float red[8];
   const int64_t m = blockIdx.x;
   const int nv = K / 8;
