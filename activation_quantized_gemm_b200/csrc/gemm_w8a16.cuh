@@ -76,7 +76,10 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
   return r;
 }
+// Every thread of the cluster.  The .aligned barrier needs each warp converged: callers may come
+// from lane-divergent code, so the warp reconverges first.
 __device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // 16 bytes at the same shared-memory offset in CTA `rank` of the cluster (distributed shared memory)

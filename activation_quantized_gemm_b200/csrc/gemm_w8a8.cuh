@@ -70,7 +70,9 @@ __device__ __forceinline__ uint32_t cta_rank_in_cluster() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
+// Every thread of the pair; the .aligned barrier needs each warp converged, so it reconverges first.
 __device__ __forceinline__ void cluster_sync() {
+  __syncwarp();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster
