@@ -1,10 +1,10 @@
-// Decode-size W8A8 GEMMs (M <= 64 tokens) for both schemes of "DeepSeek R1 INT8 quantization
+// Decode-size W8A8 GEMMs (M <= 128 tokens) for both schemes of "DeepSeek R1 INT8 quantization
 // practice on SGLang", section 2.3.  At these sizes the weights dominate the traffic, so the kernel
 // is built to stream them once from HBM:
 //
 // "Swap-AB" tcgen05.mma.kind::i8 (K = 32 per instruction): the 128 weight rows of a tile are the
 // MMA's M dimension, read by the tensor core straight from the TMA-staged 128B-swizzled shared
-// memory, and the (padded) tokens are its N dimension, so a batch of 1..64 tokens still fills the
+// memory, and the (padded) tokens are its N dimension, so a batch of 1..128 tokens still fills the
 // 128-row tensor-core tile.  The thread-block cluster of a tile splits K; its CTAs reduce-scatter
 // their partial tiles through distributed shared memory (no global scratch).
 //   warps 0..3  epilogue: thread = weight row (TMEM lane).  Channel-wise: the exact int32 dot
@@ -13,7 +13,8 @@
 //               partial sums are folded into fp32 running sums with sx[m][kb] * sw[n/128][kb].
 //   warp 4      TMA producer: weight slab [128 rows x 128 K] + activation slab [MP x 128 K].
 //   warp 5      TMEM allocation and MMA issue (4 x tcgen05.mma per slab).
-// Two CTAs share an SM (rings of 4..6 stages each); the launch keeps all CTAs in one wave.
+// Two CTAs share an SM for up to 64 tokens (rings of 4..6 stages each), one CTA for 128 (TMEM and
+// registers); the launch keeps all CTAs in one wave.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -23,7 +24,7 @@
 
 namespace i8q {
 
-constexpr int W8A8_SMALL_MAX_M = 64;
+constexpr int W8A8_SMALL_MAX_M = 128;
 
 // CPS CTAs share an SM; the stage ring fills the rest of its shared memory: under full streaming
 // load a weight slab takes about 2 us to arrive, so an SM needs of the order of 100 KB in flight.
@@ -34,7 +35,8 @@ struct W8A8SmallCfg {
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
   static constexpr int NBUF = BLOCKWISE ? 4 : 1;          // slab accumulators in TMEM
   static constexpr int TMEM_NEED = NBUF * MP;
-  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : 256;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
+  static_assert(CPS * TMEM_COLS <= 512, "TMEM of the CTAs sharing an SM");
   static constexpr int NUM_THREADS = 192;
   static constexpr int BAR_BYTES = 512;
   static constexpr int RING_BYTES = 4 * 2 * MP * 4;      // block-wise scale-product rings, one per epilogue warp
@@ -44,7 +46,7 @@ struct W8A8SmallCfg {
   static constexpr int STAGES_FIT = (BUDGET - FIXED_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT < 16 ? STAGES_FIT : 16;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + FIXED_BYTES;
-  static_assert(MP == 16 || MP == 32 || MP == 64, "MMA N");
+  static_assert(MP == 16 || MP == 32 || MP == 64 || MP == 128, "MMA N");
   static_assert(CPS == 1 || CPS == 2, "CTAs per SM");
   static_assert(STAGES >= 4, "stage ring");
   static_assert(MP * 128 * 4 <= STAGES * STAGE_BYTES, "reduction tile must fit in the stage buffers");

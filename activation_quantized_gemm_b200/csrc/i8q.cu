@@ -319,7 +319,7 @@ static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args
 template <int MP, bool BLOCKWISE, bool F32, bool DBG>
 static i8q_status launch_w8a8_small_mp(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms,
                                        cudaStream_t s) {
-  constexpr int CPS = 2;
+  constexpr int CPS = MP <= 64 ? 2 : 1;   // 128 tokens: one CTA per SM (TMEM and registers)
   using C = W8A8SmallCfg<MP, BLOCKWISE, CPS>;
   auto kern = k_gemm_w8a8_small<MP, BLOCKWISE, CPS, F32, DBG>;
   static std::once_flag once;
@@ -374,7 +374,8 @@ template <bool BLOCKWISE, bool F32, bool DBG>
 static i8q_status launch_w8a8_any(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms, cudaStream_t s) {
   if (a.M <= 16) return launch_w8a8_small_mp<16, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
   if (a.M <= 32) return launch_w8a8_small_mp<32, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
-  if (a.M <= W8A8_SMALL_MAX_M) return launch_w8a8_small_mp<64, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
+  if (a.M <= 64) return launch_w8a8_small_mp<64, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
+  if (a.M <= W8A8_SMALL_MAX_M) return launch_w8a8_small_mp<128, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
   if constexpr (!BLOCKWISE) {
     switch (channel_tile_n(a.M, a.N, sms)) {
       case 224: return launch_w8a8<224, false, F32, DBG>(xq, wq, a, sms, s);

@@ -20,8 +20,10 @@ SHAPES = [(1, 8, 128), (16, 256, 512), (7, 200, 384), (130, 264, 1024), (300, 52
           # 1..8 CTAs with slab counts that do not divide evenly, ragged last weight tile
           (17, 136, 896), (33, 520, 1152), (64, 1032, 4096), (48, 8, 256), (2, 2056, 1920),
           (65, 264, 1024),
+          # decode kernel with 128-token padding (65..128 tokens, one CTA per SM)
+          (100, 1032, 1536), (128, 264, 4096),
           # channel-wise pair-tile widths 224 and 256 (chosen by wave fill; smaller shapes take 192)
-          (100, 16384, 256), (130, 18944, 256)]
+          (200, 16384, 256), (130, 18944, 256)]
 
 
 @pytest.fixture(scope="module")
