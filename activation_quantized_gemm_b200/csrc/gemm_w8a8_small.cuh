@@ -233,13 +233,29 @@ __global__ void __launch_bounds__(192, CPS)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[b]);
           }
+          // int32 partial P (|P| <= 127^2 * 128 < 2^22) -> exact float.  Up to 64 tokens: the integer
+          // add puts P into the mantissa of 1.5 * 2^23 (the bit pattern of 12582912 + P) and a packed
+          // subtract removes the offset (full-rate ALU and FMA pipes rather than the conversion
+          // unit); at 128 tokens the register budget favours the plain conversion (measured).
 #pragma unroll
           for (int i = 0; i < CH; i += 4) {
             const float4 q = *reinterpret_cast<const float4*>(slot + c * CH + i);
-            sum[c * CH + i + 0] = fmaf(__int2float_rn((int)r[i + 0]), q.x, sum[c * CH + i + 0]);
-            sum[c * CH + i + 1] = fmaf(__int2float_rn((int)r[i + 1]), q.y, sum[c * CH + i + 1]);
-            sum[c * CH + i + 2] = fmaf(__int2float_rn((int)r[i + 2]), q.z, sum[c * CH + i + 2]);
-            sum[c * CH + i + 3] = fmaf(__int2float_rn((int)r[i + 3]), q.w, sum[c * CH + i + 3]);
+            float p[4];
+            if constexpr (MP <= 64) {
+              const float2 nb = make_float2(-12582912.0f, -12582912.0f);
+              const float2 p01 = __fadd2_rn(make_float2(__uint_as_float(r[i + 0] + 0x4B400000u),
+                                                        __uint_as_float(r[i + 1] + 0x4B400000u)), nb);
+              const float2 p23 = __fadd2_rn(make_float2(__uint_as_float(r[i + 2] + 0x4B400000u),
+                                                        __uint_as_float(r[i + 3] + 0x4B400000u)), nb);
+              p[0] = p01.x; p[1] = p01.y; p[2] = p23.x; p[3] = p23.y;
+            } else {
+#pragma unroll
+              for (int t = 0; t < 4; ++t) p[t] = __int2float_rn((int)r[i + t]);
+            }
+            sum[c * CH + i + 0] = fmaf(p[0], q.x, sum[c * CH + i + 0]);
+            sum[c * CH + i + 1] = fmaf(p[1], q.y, sum[c * CH + i + 1]);
+            sum[c * CH + i + 2] = fmaf(p[2], q.z, sum[c * CH + i + 2]);
+            sum[c * CH + i + 3] = fmaf(p[3], q.w, sum[c * CH + i + 3]);
           }
           if constexpr (DEBUG) {
             if (n < N) {

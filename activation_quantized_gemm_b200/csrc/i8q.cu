@@ -212,12 +212,13 @@ static int decode_splits(int64_t tiles, int64_t KB, int sms, int per_sm) {
   return s;
 }
 
-// Split-K factor of the decode-size W8A8 GEMM: the largest cluster size s in 1..8 (and <= K / 128)
+// Split-K factor of the decode-size W8A8 GEMM: the largest cluster size s in 1..4 (and <= K / 128)
 // whose tiles x s CTAs are all co-resident (CPS per SM), so that as many CTAs as fit stream weights
-// at once, in one wave.
+// at once, in one wave.  Clusters stay at 4 CTAs or fewer: larger ones did not all find room while
+// the quantizer that precedes the GEMM still held some SMs (dependent launch), leaving a tail.
 static int w8a8_small_splits(int64_t tiles, int64_t KB, int sms, int cps) {
   int s = 1;
-  while (s < 8 && s < KB && tiles * (s + 1) <= (int64_t)sms * cps) ++s;
+  while (s < 4 && s < KB && tiles * (s + 1) <= (int64_t)sms * cps) ++s;
   return s;
 }
 
