@@ -7,12 +7,13 @@
 // memory, and the (padded) tokens are its N dimension, so a batch of 1..128 tokens still fills the
 // 128-row tensor-core tile.  The thread-block cluster of a tile splits K; its CTAs reduce-scatter
 // their partial tiles through distributed shared memory (no global scratch).
-//   warps 0..3  epilogue: thread = weight row (TMEM lane).  Channel-wise: the exact int32 dot
+//   warps 0..3  epilogue (0..7 at 128 tokens, two token halves per TMEM lane quarter): thread =
+//               weight row (TMEM lane).  Channel-wise: the exact int32 dot
 //               products are read once at the end, summed exactly over the cluster, then scaled by
 //               sx[m] * sw[n].  Block-wise: each 128-K slab has its own TMEM accumulator; its int32
 //               partial sums are folded into fp32 running sums with sx[m][kb] * sw[n/128][kb].
-//   warp 4      TMA producer: weight slab [128 rows x 128 K] + activation slab [MP x 128 K].
-//   warp 5      TMEM allocation and MMA issue (4 x tcgen05.mma per slab).
+//   next warp   TMA producer: weight slab [128 rows x 128 K] + activation slab [MP x 128 K].
+//   last warp   TMEM allocation and MMA issue (4 x tcgen05.mma per slab).
 // Two CTAs share an SM for up to 64 tokens (rings of 4..6 stages each), one CTA for 128 (TMEM and
 // registers); the launch keeps all CTAs in one wave.
 #pragma once
@@ -37,9 +38,13 @@ struct W8A8SmallCfg {
   static constexpr int TMEM_NEED = NBUF * MP;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
   static_assert(CPS * TMEM_COLS <= 512, "TMEM of the CTAs sharing an SM");
-  static constexpr int NUM_THREADS = 192;
+  // epilogue warps: 4 (one per TMEM lane quarter), or 8 at 128 tokens (two column halves per
+  // quarter) so that the per-slab fold of 128 columns is split over twice the threads
+  static constexpr int EW = MP >= 128 ? 8 : 4;
+  static constexpr int MPW = MP / (EW / 4);              // token columns per epilogue thread
+  static constexpr int NUM_THREADS = 32 * (EW + 2);      // + TMA warp + MMA warp
   static constexpr int BAR_BYTES = 512;
-  static constexpr int RING_BYTES = 4 * 2 * MP * 4;      // block-wise scale-product rings, one per epilogue warp
+  static constexpr int RING_BYTES = EW * 2 * MPW * 4;    // block-wise scale-product rings, one per epilogue warp
   static constexpr int FIXED_BYTES = BAR_BYTES + RING_BYTES + 1024;   // + 1024-byte alignment slack
   static constexpr int SM_SMEM = 233472, CTA_RESERVED = 1024, CTA_MAX = 232448;
   static constexpr int BUDGET = (SM_SMEM / CPS - CTA_RESERVED) < CTA_MAX ? (SM_SMEM / CPS - CTA_RESERVED) : CTA_MAX;
@@ -71,11 +76,12 @@ __device__ __forceinline__ void tmem_ld_ch(uint32_t taddr, uint32_t (&r)[CH]) {
 }
 
 template <int MP, bool BLOCKWISE, int CPS, bool OUT_F32, bool DEBUG>
-__global__ void __launch_bounds__(192, CPS)
+__global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS, CPS)
     k_gemm_w8a8_small(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                       const W8A8Args args) {
   using C = W8A8SmallCfg<MP, BLOCKWISE, CPS>;
-  constexpr int CH = MP < 32 ? MP : 32;   // TMEM columns per load
+  constexpr int EW = C::EW, MPW = C::MPW;
+  constexpr int CH = MPW < 32 ? MPW : 32;   // TMEM columns per load
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
@@ -99,21 +105,21 @@ __global__ void __launch_bounds__(192, CPS)
   // its first weight slabs, so that the weight stream starts as early as possible.  It lets the next
   // kernel launch early in turn (that kernel waits for this one the same way).
   grid_dependents_launch();
-  if (warp == 4 && lane == 0) {
+  if (warp == EW && lane == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < C::NBUF; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], EW);
     }
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
     for (int j = 0; j < nslab && j < C::STAGES; ++j) tma_prefetch_l2_2d(&tmW, (kb0 + j) * 128, n0);
   }
-  if (warp == 5) {
+  if (warp == EW + 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -124,15 +130,15 @@ __global__ void __launch_bounds__(192, CPS)
   grid_dependency_wait();
 
   // per-thread results of the epilogue warps: channel: exact int32 dot products; block: fp32 sums
-  int32_t acc[MP];
-  float sum[MP];
+  int32_t acc[MPW];
+  float sum[MPW];
 #pragma unroll
-  for (int m = 0; m < MP; ++m) {
+  for (int m = 0; m < MPW; ++m) {
     acc[m] = 0;
     sum[m] = 0.f;
   }
 
-  if (warp == 4) {
+  if (warp == EW) {
     if (lane == 0) {
       uint32_t filled = 0, par = 0;
       bool ok = true;
@@ -152,7 +158,7 @@ __global__ void __launch_bounds__(192, CPS)
         for (int s = 0; s < C::STAGES; ++s)
           if (filled & (1u << s)) mbar_wait(&full[s], (par >> s) & 1u, SITE_DRAIN, nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == EW + 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_i8(128, MP);
       for (int j = 0; j < nslab; ++j) {
@@ -179,17 +185,19 @@ __global__ void __launch_bounds__(192, CPS)
       mbar_wait(done, 0, SITE_DRAIN, nullptr);
     }
   } else {
-    // epilogue: thread = weight row n0 + 32 * warp + lane (TMEM lane quarter = warp)
-    const int row = warp * 32 + lane;
+    // epilogue: thread = weight row n0 + 32 * (warp % 4) + lane (TMEM lane quarter = warp % 4),
+    // token columns cb .. cb + MPW - 1
+    const int row = (warp & 3) * 32 + lane;
     const int n = n0 + row;
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    const int cb = (warp >> 2) * MPW;
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
     if constexpr (!BLOCKWISE) {
       if (nslab > 0 && warp_wait(&tfull[0], 0, SITE_TMEM_FULL, abort_flag)) {
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < MP / CH; ++c) {
+        for (int c = 0; c < MPW / CH; ++c) {
           uint32_t r[CH];
-          tmem_ld_ch<CH>(tmem + lane_addr + c * CH, r);
+          tmem_ld_ch<CH>(tmem + lane_addr + cb + c * CH, r);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < CH; ++i) acc[c * CH + i] = (int32_t)r[i];
@@ -200,35 +208,35 @@ __global__ void __launch_bounds__(192, CPS)
       // shared memory: lane l loads token l (and l + 32) of slab j + 1 while slab j is folded, so
       // the global-load latency is hidden behind one slab of streaming.
       const float* swrow = args.sw + (int64_t)(n0 / 128) * KB;
-      float* ring = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES) + warp * 2 * MP;
-      constexpr int PER_LANE = (MP + 31) / 32;
+      float* ring = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES) + warp * 2 * MPW;
+      constexpr int PER_LANE = (MPW + 31) / 32;
       float nsx[PER_LANE], nsw = 0.f;
       auto load_scales = [&](int kb) {
         nsw = __ldg(swrow + kb);
 #pragma unroll
         for (int i = 0; i < PER_LANE; ++i) {
-          const int m = lane + 32 * i;
-          nsx[i] = (m < MP && m < M) ? __ldg(args.sx + (int64_t)kb * args.ld_sx + m) : 0.f;
+          const int m = cb + lane + 32 * i;
+          nsx[i] = (lane + 32 * i < MPW && m < M) ? __ldg(args.sx + (int64_t)kb * args.ld_sx + m) : 0.f;
         }
       };
       if (nslab > 0) load_scales(kb0);
       for (int j = 0; j < nslab; ++j) {
         const int b = j % C::NBUF;
         const int kb = kb0 + j;
-        float* slot = ring + (j & 1) * MP;
+        float* slot = ring + (j & 1) * MPW;
 #pragma unroll
         for (int i = 0; i < PER_LANE; ++i)
-          if (lane + 32 * i < MP) slot[lane + 32 * i] = nsx[i] * nsw;
+          if (lane + 32 * i < MPW) slot[lane + 32 * i] = nsx[i] * nsw;
         __syncwarp();
         if (j + 1 < nslab) load_scales(kb + 1);
         if (!warp_wait(&tfull[b], (j / C::NBUF) & 1, SITE_TMEM_FULL, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < MP / CH; ++c) {
+        for (int c = 0; c < MPW / CH; ++c) {
           uint32_t r[CH];
-          tmem_ld_ch<CH>(tmem + lane_addr + b * MP + c * CH, r);
+          tmem_ld_ch<CH>(tmem + lane_addr + b * MP + cb + c * CH, r);
           tmem_ld_wait();
-          if (c == MP / CH - 1) {
+          if (c == MPW / CH - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[b]);
@@ -241,7 +249,7 @@ __global__ void __launch_bounds__(192, CPS)
           for (int i = 0; i < CH; i += 4) {
             const float4 q = *reinterpret_cast<const float4*>(slot + c * CH + i);
             float p[4];
-            if constexpr (MP <= 64) {
+            if constexpr (MPW <= 64) {
               const float2 nb = make_float2(-12582912.0f, -12582912.0f);
               const float2 p01 = __fadd2_rn(make_float2(__uint_as_float(r[i + 0] + 0x4B400000u),
                                                         __uint_as_float(r[i + 1] + 0x4B400000u)), nb);
@@ -261,7 +269,7 @@ __global__ void __launch_bounds__(192, CPS)
             if (n < N) {
 #pragma unroll
               for (int i = 0; i < CH; ++i)
-                if (c * CH + i < M) args.dbg[((int64_t)(c * CH + i) * N + n) * KB + kb] = (int32_t)r[i];
+                if (cb + c * CH + i < M) args.dbg[((int64_t)(cb + c * CH + i) * N + n) * KB + kb] = (int32_t)r[i];
             }
           }
         }
@@ -281,18 +289,20 @@ __global__ void __launch_bounds__(192, CPS)
       reinterpret_cast<uint16_t*>(args.y)[(int64_t)m * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
   };
   if (nrank == 1) {
-    if (warp < 4) {
-      const int n = n0 + warp * 32 + lane;
+    if (warp < EW) {
+      const int n = n0 + (warp & 3) * 32 + lane;
+      const int cb = (warp >> 2) * MPW;
       if (n < N) {
         const float swn = BLOCKWISE ? 0.f : __ldg(args.sw + n);
 #pragma unroll
-        for (int m = 0; m < MP; ++m) {
+        for (int i = 0; i < MPW; ++i) {
+          const int m = cb + i;
           if (m < mlim) {
             if constexpr (BLOCKWISE) {
-              write_out(n, m, sum[m]);
+              write_out(n, m, sum[i]);
             } else {
-              write_out(n, m, __int2float_rn(acc[m]) * (__ldg(args.sx + m) * swn));
-              if constexpr (DEBUG) args.dbg[(int64_t)m * N + n] = acc[m];
+              write_out(n, m, __int2float_rn(acc[i]) * (__ldg(args.sx + m) * swn));
+              if constexpr (DEBUG) args.dbg[(int64_t)m * N + n] = acc[i];
             }
           }
         }
@@ -302,15 +312,16 @@ __global__ void __launch_bounds__(192, CPS)
     // partial tiles in [MP / 4][128 rows] of 4 x 32-bit (the stage buffers are idle now); CTA `rank`
     // owns rows [128 * rank / nrank, 128 * (rank + 1) / nrank) and sums them over all ranks in rank order
     uint4* red = reinterpret_cast<uint4*>(smem);
-    if (warp < 4) {
-      const int row = warp * 32 + lane;
+    if (warp < EW) {
+      const int row = (warp & 3) * 32 + lane;
+      const int c4 = (warp >> 2) * (MPW / 4);
 #pragma unroll
-      for (int m4 = 0; m4 < MP / 4; ++m4) {
+      for (int m4 = 0; m4 < MPW / 4; ++m4) {
         if constexpr (BLOCKWISE)
-          red[m4 * 128 + row] = make_uint4(__float_as_uint(sum[4 * m4]), __float_as_uint(sum[4 * m4 + 1]),
-                                           __float_as_uint(sum[4 * m4 + 2]), __float_as_uint(sum[4 * m4 + 3]));
+          red[(c4 + m4) * 128 + row] = make_uint4(__float_as_uint(sum[4 * m4]), __float_as_uint(sum[4 * m4 + 1]),
+                                                  __float_as_uint(sum[4 * m4 + 2]), __float_as_uint(sum[4 * m4 + 3]));
         else
-          red[m4 * 128 + row] = make_uint4(acc[4 * m4], acc[4 * m4 + 1], acc[4 * m4 + 2], acc[4 * m4 + 3]);
+          red[(c4 + m4) * 128 + row] = make_uint4(acc[4 * m4], acc[4 * m4 + 1], acc[4 * m4 + 2], acc[4 * m4 + 3]);
       }
     }
     cluster_sync_all();
@@ -366,7 +377,7 @@ __global__ void __launch_bounds__(192, CPS)
     cluster_sync_all();   // no CTA leaves while its shared memory may still be read
   }
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == EW + 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace i8q
