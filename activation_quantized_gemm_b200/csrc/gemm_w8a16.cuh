@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
 
   // ---- output.  Without a split the epilogue threads write their rows directly.  With a split,
   // every CTA publishes its fp32 partial tile ([128 rows][MP] in shared memory) and CTA `rank` sums
-  // rows r with r % nrank == rank over all ranks, in rank order, 4 tokens per 16-byte load.
+  // its block of rows over all ranks, in rank order, 4 tokens per 16-byte load.
   tc_fence_before();
   __syncthreads();
   const int mlim = args.M < MP ? args.M : MP;
@@ -364,11 +364,14 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
         red[row * (MP / 4) + m4] = make_float4(sum[4 * m4], sum[4 * m4 + 1], sum[4 * m4 + 2], sum[4 * m4 + 3]);
     }
     cluster_sync_all();
-    const int owned = (W8A16_BN - (int)rank + (int)nrank - 1) / (int)nrank;   // rows rank + i * nrank
+    // CTA `rank` owns a contiguous block of rows; consecutive threads take consecutive rows of one
+    // 4-token group, so that a warp's fp16 stores are contiguous.
+    const int rb0 = W8A16_BN * (int)rank / (int)nrank, rb1 = W8A16_BN * ((int)rank + 1) / (int)nrank;
+    const int owned = rb1 - rb0;
     const int items = owned * (MP / 4);
     for (int e = threadIdx.x; e < items; e += C::NUM_THREADS) {
-      const int i = e / (MP / 4), m4 = e - (e / (MP / 4)) * (MP / 4);
-      const int row = (int)rank + i * (int)nrank;
+      const int m4 = e / owned;
+      const int row = rb0 + (e - m4 * owned);
       const uint32_t la = smem_u32(&red[row * (MP / 4) + m4]);
       float4 part[8];
 #pragma unroll

@@ -199,16 +199,16 @@ static i8q_status launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned blo
 }
 
 // ------------------------------------------------------------------ W8A16 launch ------------
-// Split-K factor of the decode-size (weight-streaming) GEMMs: the smallest cluster size s in 1..8
-// that gives at least three quarters of the SMs a CTA (one CTA streams about 60 GB/s, so about 110
-// of them saturate HBM), without going past one wave of co-resident CTAs (about 95% of the SMs'
-// CTA slots: cluster placement within GPCs leaves a few SMs unused).  Every extra wave would pay
-// the per-CTA start-up and pipeline-fill latency again.
+// Split-K factor of the W8A16 GEMM: the largest cluster size s in 1..8 (and <= K / 128) whose
+// tiles x s CTAs stay within one wave of co-resident CTAs (about 95% of the SMs' CTA slots: cluster
+// placement within GPCs leaves a few SMs unused).  Filling both CTA slots of an SM matters: one CTA
+// streams weights well below an SM's share of HBM bandwidth (measured: N = 4096, K = 12288, 16
+// tokens takes 24 us at s = 4 and 16.5 us at s = 8), while an extra wave would pay the per-CTA
+// start-up and pipeline-fill latency again.
 static int decode_splits(int64_t tiles, int64_t KB, int sms, int per_sm) {
   const int64_t slots = (int64_t)(sms * 95 / 100) * per_sm;
-  const int64_t target = (int64_t)sms * 3 / 4;
   int s = 1;
-  while (s < 8 && s < KB && tiles * s < target && tiles * (s + 1) <= slots) ++s;
+  while (s < 8 && s < KB && tiles * (s + 1) <= slots) ++s;
   return s;
 }
 
