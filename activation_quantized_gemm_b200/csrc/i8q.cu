@@ -439,7 +439,7 @@ i8q_status i8q_quant_act_token_group(const uint16_t* x, int64_t M, int64_t K, in
   i8q_status st = current_device(&sms);
   if (st) return st;
   const int64_t KB = K / 128;
-  constexpr int U = 2;
+  constexpr int U = 1;   // one warp step per item: 63 registers, four CTAs per SM (U = 2: 99, two)
   const int64_t items = M * cdiv(cdiv(KB, 8), U);
   I8Q_REQUIRE(items < ((int64_t)1 << 31), I8Q_ERR_SHAPE);
   int64_t blocks = cdiv(items, 8);
