@@ -11,17 +11,22 @@
 // its N dimension, so a decode batch of 1..64 tokens still fills the 128-row tensor-core tile.
 //   warps 0..3   epilogue: thread = weight row; per slab, sum[m] += partial[m] * s[n][g].
 //   warps 4..7   converters: int8 slab (shared memory) -> exact f16 operand written straight into
-//                TMEM with tcgen05.st (NA operand buffers); the MMA reads its A operand from TMEM,
-//                so shared memory only carries the TMA-staged int8 weights and f16 activations.
-//   warp 8       TMA: lane 0 fills the int8 weight ring ([128 rows x 128 K] slabs, 128B swizzle,
-//                released by the converters), lane 1 the f16 activation ring ([MP x 128 K] as two
-//                64-element halves, 128B swizzle, released by the MMA).
+//                TMEM with tcgen05.st; the MMA reads its A operand from TMEM, so shared memory only
+//                carries the TMA-staged int8 weights and f16 activations.
+//   warp 8       TMA: lane 0 streams the int8 weight ring ([128 rows x 128 K] slabs, 128B swizzle;
+//                a stage is released as soon as the converters have read it), lane 1 the f16
+//                activation ring ([MP x 128 K] as two 64-element halves, released by the MMA),
+//                lane 2 reports landed activation slabs to the MMA (see below).
 //   warp 9       TMEM allocation and MMA issue: 8 x tcgen05.mma.kind::f16 (K = 16) per slab.
-// For decode batches of up to 32 tokens two CTAs share an SM (256 TMEM columns each), so that a
-// single wave holds every CTA of the split-K grid.
-// Small-N MMAs have a long latency compared with their work, so consecutive MMAs do not wait on
-// each other: a slab's 8 k-steps are spread over NACC independent TMEM accumulators (each folded
-// into the running sum by the epilogue), and NBUF slabs are in flight in a ring of TMEM buffers.
+// For decode batches of up to 32 tokens two CTAs share an SM (256 TMEM columns each).
+// The MMA thread is the serial part of the pipeline and every mbarrier probe it makes costs about
+// as much as two small MMAs, so each slab costs it one wait and two commits:
+//   * TMEM holds R "slots" (an f16 operand buffer + the slab's fp32 accumulator).  ready[slot]
+//     completes when the 4 converter warps have written the operand, the 4 epilogue warps have read
+//     out the accumulator's previous slab (they pre-arrive once per slot at start) and the
+//     activation slab has landed (warp 8 lane 2 observes the TMA barrier and arrives).
+//   * mdone[slot] (commit) tells the epilogue the accumulator is ready and the converters that the
+//     operand buffer may be overwritten; xempty (commit) releases the activation stage.
 // Split-K: the CTAs of one thread-block cluster take disjoint slab ranges of the same 128 rows and
 // reduce-scatter their fp32 partial tiles through distributed shared memory (each CTA sums its
 // share of the rows over all ranks, in rank order, and writes fp16).
@@ -38,26 +43,25 @@ constexpr int W8A16_BN = 128;   // weight rows per tile (MMA M)
 
 template <int MP>
 struct W8A16Cfg {
-  static constexpr int W_BYTES = W8A16_BN * 128;        // int8 slab
-  static constexpr int X_HALF = MP * 128;               // one 64-element half of the f16 slab
+  static constexpr int W_BYTES = W8A16_BN * 128;         // int8 weight slab
+  static constexpr int X_HALF = MP * 128;                // one 64-element half of the f16 slab
   static constexpr int X_BYTES = 2 * X_HALF;
-  static constexpr int CTAS_PER_SM = MP <= 32 ? 2 : 1;  // two CTAs share an SM's TMEM and smem
-  static constexpr int W_STAGES = CTAS_PER_SM == 2 ? 5 : 8;   // weight ring (freed after conversion)
-  static constexpr int X_STAGES = MP <= 16 ? 4 : (MP <= 32 ? 3 : 4);   // activation ring (freed by the MMA)
-  static constexpr int A_COLS = 64;                     // 128 K f16 values = 64 packed 32-bit columns
-  static constexpr int NACC = 2;                        // independent accumulators per slab
-  static constexpr int SLAB_COLS = NACC * MP;           // TMEM columns of one slab's partials
+  static constexpr int CTAS_PER_SM = MP <= 32 ? 2 : 1;   // two CTAs share an SM's TMEM and smem
   static constexpr int TMEM_COLS = CTAS_PER_SM == 2 ? 256 : 512;
-  static constexpr int NA = MP <= 16 ? 3 : 2;           // f16 operand buffers (in TMEM)
-  static constexpr int NBUF_FIT = (TMEM_COLS - NA * A_COLS) / SLAB_COLS;
-  static constexpr int NBUF = NBUF_FIT < 4 ? NBUF_FIT : 4;
-  static constexpr int NUM_THREADS = 320;               // warps 0-3 epilogue, 4-7 converters, 8 TMA, 9 MMA
+  static constexpr int A_COLS = 64;                      // 128 K f16 values = 64 packed 32-bit columns
+  static constexpr int SLOT_COLS = A_COLS + MP;          // operand buffer + accumulator
+  static constexpr int R_FIT = TMEM_COLS / SLOT_COLS;
+  static constexpr int R = R_FIT < 4 ? R_FIT : 4;        // TMEM slots
+  static constexpr int W_STAGES = MP <= 16 ? 5 : (MP <= 32 ? 4 : 8);   // weight ring (freed after conversion)
+  static constexpr int X_STAGES = MP <= 16 ? 6 : 5;      // activation ring (freed by the MMA)
+  static constexpr int NUM_THREADS = 320;                // warps 0-3 epilogue, 4-7 converters, 8 TMA, 9 MMA
   static constexpr int RING_BYTES = W_STAGES * W_BYTES + X_STAGES * X_BYTES;
   static constexpr int SMEM_BYTES = RING_BYTES + 512 + 1024;
-  static_assert(NBUF >= 2, "at least two slabs in flight");
-  static_assert(MP * W8A16_BN * 4 <= RING_BYTES, "reduction tile must fit in the ring buffers");
-  static_assert(MP % 4 == 0, "tokens are reduced four at a time");
-  static_assert(SMEM_BYTES * CTAS_PER_SM <= 229376, "shared memory");
+  static_assert(R >= 2 && X_STAGES > R, "pipeline depth");
+  static_assert(X_BYTES % 1024 == 0, "128B-swizzled TMA boxes need 1024-byte alignment");
+  static_assert(MP * W8A16_BN * 4 <= RING_BYTES, "reduction tile must fit in the ring");
+  static_assert(MP % 16 == 0, "MMA N and the 16-column TMEM loads");
+  static_assert(CTAS_PER_SM * (SMEM_BYTES + 1024) <= 233472, "shared memory per SM");
 };
 
 struct W8A16Args {
@@ -134,19 +138,18 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
     k_gemm_w8a16(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const W8A16Args args) {
   using C = W8A16Cfg<MP>;
+  constexpr int R = C::R;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sW = smem;                                       // W_STAGES x int8 weight slab
-  uint8_t* sX = smem + C::W_STAGES * C::W_BYTES;            // X_STAGES x f16 activation slab halves
+  uint8_t* sX = smem + C::W_STAGES * C::W_BYTES;            // X_STAGES x f16 activation slab
   uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES);
   uint64_t* wempty = wfull + C::W_STAGES;
   uint64_t* xfull = wempty + C::W_STAGES;
   uint64_t* xempty = xfull + C::X_STAGES;
-  uint64_t* afull = xempty + C::X_STAGES;
-  uint64_t* aempty = afull + C::NA;
-  uint64_t* tfull = aempty + C::NA;
-  uint64_t* tempty = tfull + C::NBUF;
-  uint64_t* done = tempty + C::NBUF;
+  uint64_t* ready = xempty + C::X_STAGES;
+  uint64_t* mdone = ready + R;
+  uint64_t* done = mdone + R;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -167,13 +170,9 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
       mbar_init(&xfull[s], 1);
       mbar_init(&xempty[s], 1);   // the MMA's commit
     }
-    for (int a = 0; a < C::NA; ++a) {
-      mbar_init(&afull[a], 4);
-      mbar_init(&aempty[a], 1);
-    }
-    for (int b = 0; b < C::NBUF; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+    for (int r = 0; r < R; ++r) {
+      mbar_init(&ready[r], 9);    // 4 converter warps + 4 epilogue warps + the activation reporter
+      mbar_init(&mdone[r], 1);    // the MMA's commit
     }
     mbar_init(done, 1);
     *abort_flag = 0;
@@ -200,9 +199,9 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
   for (int m = 0; m < MP; ++m) sum[m] = 0.f;
 
   if (warp == 8) {
-    // lane 0 feeds the weight ring (waits only for the converters), lane 1 the activation ring
-    // (waits only for the MMA); the two rings run ahead independently.
     if (lane < 2) {
+      // lane 0 feeds the weight ring (waits only for the converters), lane 1 the activation ring
+      // (waits only for the MMA); the two rings run ahead independently.
       const bool is_w = lane == 0;
       const int nst = is_w ? C::W_STAGES : C::X_STAGES;
       uint64_t* fullb = is_w ? wfull : xfull;
@@ -226,57 +225,59 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
         filled |= 1u << st;
         par = (par & ~(1u << st)) | (ph << st);
       }
-      if (!ok)
+      if (!ok)   // let every copy in flight land before the CTA can exit
         for (int st = 0; st < nst; ++st)
           if (filled & (1u << st)) mbar_wait(&fullb[st], (par >> st) & 1u, SITE_DRAIN, nullptr);
+    } else if (lane == 2) {
+      // activation reporter: one arrival on the slab's slot once its activations have landed, so
+      // that the MMA thread needs a single wait per slab.  The activation ring runs further ahead
+      // than the slots, so an arrival for slab j also waits until the slot's previous slab (j - R)
+      // has been issued, i.e. its ready phase is over (an earlier arrival would count towards it).
+      for (int j = 0; j < nslab; ++j) {
+        const int r = j % R;
+        if (!mbar_wait(&xfull[j % C::X_STAGES], (j / C::X_STAGES) & 1, SITE_FULL, abort_flag)) break;
+        if (j >= R && !mbar_wait(&mdone[r], ((j / R) & 1) ^ 1, SITE_CONVERT, abort_flag)) break;
+        mbar_arrive(&ready[r]);
+      }
     }
   } else if (warp == 9) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16(W8A16_BN, MP);
       for (int j = 0; j < nslab; ++j) {
-        const int sx_ = j % C::X_STAGES;
-        const uint32_t px = (j / C::X_STAGES) & 1;
-        const int a = j % C::NA;
-        const uint32_t pa = (j / C::NA) & 1;
-        const int b = j % C::NBUF;
-        const uint32_t pb = (j / C::NBUF) & 1;
-        if (!mbar_wait(&tempty[b], pb ^ 1, SITE_TMEM_EMPTY, abort_flag)) break;
-        if (!mbar_wait(&afull[a], pa, SITE_CONVERT, abort_flag)) break;
-        if (!mbar_wait(&xfull[sx_], px, SITE_FULL, abort_flag)) break;
+        const int xs = j % C::X_STAGES;
+        const int r = j % R;
+        if (!mbar_wait(&ready[r], (j / R) & 1, SITE_CONVERT, abort_flag)) break;
         tc_fence_after();
-        const uint32_t a0 = tmem + a * C::A_COLS;                       // operand columns
-        const uint32_t x0 = smem_u32(sX + sx_ * C::X_BYTES);
-        const uint32_t d0 = tmem + C::NA * C::A_COLS + b * C::SLAB_COLS;  // accumulator columns
+        const uint32_t a0 = tmem + r * C::A_COLS;                        // operand columns
+        const uint32_t d0 = tmem + R * C::A_COLS + r * MP;               // accumulator columns
+        const uint32_t x0 = smem_u32(sX + xs * C::X_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t h = kk >> 2, off = (kk & 3) * 32;
-          mma_f16_ts(d0 + (kk % C::NACC) * MP, a0 + kk * 8, sw128_kmajor_desc(x0 + h * C::X_HALF + off), idesc,
-                     kk >= C::NACC);
+          mma_f16_ts(d0, a0 + kk * 8, sw128_kmajor_desc(x0 + h * C::X_HALF + off), idesc, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&xempty[sx_]);
-        tc_commit(&aempty[a]);
-        tc_commit(&tfull[b]);
+        tc_commit(&mdone[r]);
+        tc_commit(&xempty[xs]);
       }
       tc_commit(done);
       mbar_wait(done, 0, SITE_DRAIN, nullptr);
     }
   } else if (warp >= 4 && warp < 8) {
     // converters: warp w owns weight rows 32 (w % 4) .. + 31 (its TMEM lane quarter); each thread
-    // writes the exact f16 values of its row's 128 K into the operand's TMEM columns (two f16 per
+    // writes the exact f16 values of its row's 128 K into the slot's operand columns (two f16 per
     // 32-bit column, K order).
     const int q = warp & 3;
-    const int r = q * 32 + lane;
-    const int sw = r & 7;
+    const int row = q * 32 + lane;
+    const int sw = row & 7;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     for (int j = 0; j < nslab; ++j) {
-      const int sw_ = j % C::W_STAGES;
-      const uint32_t pw = (j / C::W_STAGES) & 1;
-      const int a = j % C::NA;
-      const uint32_t pa = (j / C::NA) & 1;
-      if (!warp_wait(&wfull[sw_], pw, SITE_FULL, abort_flag)) break;
-      if (!warp_wait(&aempty[a], pa ^ 1, SITE_CONVERT, abort_flag)) break;
+      const int st = j % C::W_STAGES;
+      const int r = j % R;
+      if (!warp_wait(&wfull[st], (j / C::W_STAGES) & 1, SITE_FULL, abort_flag)) break;
+      // the operand buffer is free once the MMAs of the slot's previous slab have completed
+      if (j >= R && !warp_wait(&mdone[r], ((j / R) & 1) ^ 1, SITE_CONVERT, abort_flag)) break;
       tc_fence_after();
-      const uint8_t* wrow = sW + sw_ * C::W_BYTES + r * 128;
+      const uint8_t* wrow = sW + st * C::W_BYTES + row * 128;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t o[32];
@@ -288,14 +289,14 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
           i8x4_to_f16x4(v.z, o[8 * i + 4], o[8 * i + 5]);
           i8x4_to_f16x4(v.w, o[8 * i + 6], o[8 * i + 7]);
         }
-        tmem_st32(tmem + lane_addr + a * C::A_COLS + h * 32, o);
+        tmem_st32(tmem + lane_addr + r * C::A_COLS + h * 32, o);
       }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&afull[a]);
-        mbar_arrive(&wempty[sw_]);
+        mbar_arrive(&ready[r]);
+        mbar_arrive(&wempty[st]);
       }
     }
   } else if (warp < 4) {
@@ -304,39 +305,27 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
     const int n = n0 + q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     const int G = KB;
+    if (lane == 0)
+      for (int r = 0; r < R; ++r) mbar_arrive(&ready[r]);   // every accumulator starts out free
     float sc_next = (n < N && nslab > 0) ? __half2float(__ushort_as_half(__ldg(args.s + (int64_t)n * G + kb0))) : 0.f;
     for (int j = 0; j < nslab; ++j) {
-      const int b = j % C::NBUF;
-      const uint32_t pb = (j / C::NBUF) & 1;
+      const int r = j % R;
       const float sc = sc_next;
       if (j + 1 < nslab && n < N) sc_next = __half2float(__ushort_as_half(__ldg(args.s + (int64_t)n * G + kb0 + j + 1)));
-      if (!warp_wait(&tfull[b], pb, SITE_TMEM_FULL, abort_flag)) break;
+      if (!warp_wait(&mdone[r], (j / R) & 1, SITE_TMEM_FULL, abort_flag)) break;
       tc_fence_after();
-      const uint32_t base = tmem + lane_addr + C::NA * C::A_COLS + b * C::SLAB_COLS;
-      // every column c of the slab holds a partial of token c % MP: fold each into the running sum
-      if constexpr (C::SLAB_COLS == 32) {
-        uint32_t p0[32];
-        tmem_ld32(base, p0);
+      const uint32_t base = tmem + lane_addr + R * C::A_COLS + r * MP;
+#pragma unroll
+      for (int c0 = 0; c0 < MP; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(base + c0, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) sum[j % MP] = fmaf(__uint_as_float(p0[j]), sc, sum[j % MP]);
-      } else {
-        static_assert(C::SLAB_COLS % 64 == 0, "slab columns");
-#pragma unroll
-        for (int c0 = 0; c0 < C::SLAB_COLS; c0 += 64) {
-          uint32_t p0[32], p1[32];
-          tmem_ld32(base + c0, p0);
-          tmem_ld32(base + c0 + 32, p1);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) sum[(c0 + j) % MP] = fmaf(__uint_as_float(p0[j]), sc, sum[(c0 + j) % MP]);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) sum[(c0 + 32 + j) % MP] = fmaf(__uint_as_float(p1[j]), sc, sum[(c0 + 32 + j) % MP]);
-        }
+        for (int i = 0; i < 16; ++i) sum[c0 + i] = fmaf(__uint_as_float(v[i]), sc, sum[c0 + i]);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[b]);
+      if (lane == 0) mbar_arrive(&ready[r]);
     }
   }
 
