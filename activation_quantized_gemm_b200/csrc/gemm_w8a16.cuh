@@ -15,16 +15,15 @@
 //                carries the TMA-staged int8 weights and f16 activations.
 //   warp 8       TMA: lane 0 streams the int8 weight ring ([128 rows x 128 K] slabs, 128B swizzle;
 //                a stage is released as soon as the converters have read it), lane 1 the f16
-//                activation ring ([MP x 128 K] as two 64-element halves, released by the MMA),
-//                lane 2 reports landed activation slabs to the MMA (see below).
+//                activation ring ([MP x 128 K] as two 64-element halves, released by the MMA).
 //   warp 9       TMEM allocation and MMA issue: 8 x tcgen05.mma.kind::f16 (K = 16) per slab.
 // For decode batches of up to 32 tokens two CTAs share an SM (256 TMEM columns each).
 // The MMA thread is the serial part of the pipeline and every mbarrier probe it makes costs about
 // as much as two small MMAs, so each slab costs it one wait and two commits:
 //   * TMEM holds R "slots" (an f16 operand buffer + the slab's fp32 accumulator).  ready[slot]
 //     completes when the 4 converter warps have written the operand, the 4 epilogue warps have read
-//     out the accumulator's previous slab (they pre-arrive once per slot at start) and the
-//     activation slab has landed (warp 8 lane 2 observes the TMA barrier and arrives).
+//     out the accumulator's previous slab (they pre-arrive once per slot at start); epilogue warp 0
+//     arrives only once the slab's activations have landed.
 //   * mdone[slot] (commit) tells the epilogue the accumulator is ready and the converters that the
 //     operand buffer may be overwritten; xempty (commit) releases the activation stage.
 // Split-K: the CTAs of one thread-block cluster take disjoint slab ranges of the same 128 rows and
@@ -171,7 +170,7 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
       mbar_init(&xempty[s], 1);   // the MMA's commit
     }
     for (int r = 0; r < R; ++r) {
-      mbar_init(&ready[r], 9);    // 4 converter warps + 4 epilogue warps + the activation reporter
+      mbar_init(&ready[r], 8);    // 4 converter warps + 4 epilogue warps
       mbar_init(&mdone[r], 1);    // the MMA's commit
     }
     mbar_init(done, 1);
@@ -228,17 +227,6 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
       if (!ok)   // let every copy in flight land before the CTA can exit
         for (int st = 0; st < nst; ++st)
           if (filled & (1u << st)) mbar_wait(&fullb[st], (par >> st) & 1u, SITE_DRAIN, nullptr);
-    } else if (lane == 2) {
-      // activation reporter: one arrival on the slab's slot once its activations have landed, so
-      // that the MMA thread needs a single wait per slab.  The activation ring runs further ahead
-      // than the slots, so an arrival for slab j also waits until the slot's previous slab (j - R)
-      // has been issued, i.e. its ready phase is over (an earlier arrival would count towards it).
-      for (int j = 0; j < nslab; ++j) {
-        const int r = j % R;
-        if (!mbar_wait(&xfull[j % C::X_STAGES], (j / C::X_STAGES) & 1, SITE_FULL, abort_flag)) break;
-        if (j >= R && !mbar_wait(&mdone[r], ((j / R) & 1) ^ 1, SITE_CONVERT, abort_flag)) break;
-        mbar_arrive(&ready[r]);
-      }
     }
   } else if (warp == 9) {
     if (lane == 0) {
@@ -305,8 +293,20 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
     const int n = n0 + q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     const int G = KB;
-    if (lane == 0)
-      for (int r = 0; r < R; ++r) mbar_arrive(&ready[r]);   // every accumulator starts out free
+    // Arrival on the slot of slab t: its accumulator is free.  Epilogue warp 0 also vouches for slab
+    // t's activations (it observes their TMA barrier first), so that the MMA thread needs a single
+    // wait per slab.  The activation ring runs further ahead than the slots, but its stage of slab t
+    // cannot be refilled before slab t's MMAs, which wait for this arrival.
+    auto free_slot = [&](int t) {
+      if (lane == 0) {
+        bool ok = true;
+        if (q == 0 && t < nslab)
+          ok = mbar_wait(&xfull[t % C::X_STAGES], (t / C::X_STAGES) & 1, SITE_FULL, abort_flag);
+        if (ok) mbar_arrive(&ready[t % R]);
+      }
+      __syncwarp();
+    };
+    for (int r = 0; r < R; ++r) free_slot(r);   // every accumulator starts out free
     float sc_next = (n < N && nslab > 0) ? __half2float(__ushort_as_half(__ldg(args.s + (int64_t)n * G + kb0))) : 0.f;
     for (int j = 0; j < nslab; ++j) {
       const int r = j % R;
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ready[r]);
+      free_slot(j + R);
     }
   }
 
