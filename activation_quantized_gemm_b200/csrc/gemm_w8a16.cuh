@@ -21,9 +21,9 @@
 // The MMA thread is the serial part of the pipeline and every mbarrier probe it makes costs about
 // as much as two small MMAs, so each slab costs it one wait and two commits:
 //   * TMEM holds R "slots" (an f16 operand buffer + the slab's fp32 accumulator).  ready[slot]
-//     completes when the 4 converter warps have written the operand, the 4 epilogue warps have read
-//     out the accumulator's previous slab (they pre-arrive once per slot at start); epilogue warp 0
-//     arrives only once the slab's activations have landed.
+//     completes when the 4 converter warps have written the operand and the 4 epilogue warps have
+//     read out the accumulator's previous slab (they pre-arrive once per slot at start); epilogue
+//     warp 0 arrives only once the slab's activations have landed.
 //   * mdone[slot] (commit) tells the epilogue the accumulator is ready and the converters that the
 //     operand buffer may be overwritten; xempty (commit) releases the activation stage.
 // Split-K: the CTAs of one thread-block cluster take disjoint slab ranges of the same 128 rows and
