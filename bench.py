@@ -60,8 +60,8 @@ MEASURED_TRAFFIC = {
     ("w8a8_block", 16384, 18432, 7168): (1824.7e6, "w8a8_block_up_m16384.md"),
     ("w8a8_block", 16, 18432, 7168): (138.08e6, "w8a8_small_block_up_m16.md"),
     ("requant", 0, 18432, 7168): (217.65e6, "requant_fp8_block_n18432_k7168.md"),
-    ("w8a16", 16, 12288, 4096): (51.29e6, "w8a16_m16_n12288_k4096.md"),
-    ("w8a16", 16, 4096, 12288): (51.58e6, "w8a16_m16_n4096_k12288.md"),
+    ("w8a16", 16, 12288, 4096): (51.30e6, "w8a16_m16_n12288_k4096.md"),
+    ("w8a16", 16, 4096, 12288): (51.55e6, "w8a16_m16_n4096_k12288.md"),
 }
 
 
