@@ -114,6 +114,42 @@ def _rotations(bytes_per_copy: int) -> int:
     return max(1, min(16, -(-2 * L2_BYTES // max(1, bytes_per_copy)) + 1))
 
 
+def describe(name: str, args) -> dict:
+    """Shapes, rotation count and the JSON `config` of a workload, from the arguments alone (no
+    device buffers): the GPU arm and the reference arm report the same config."""
+    world = getattr(args, "world", 1)
+    if name == "w8a8_channel":
+        M, N, K = args.M or 4096, 7168, 2048
+        R = _rotations(M * K * 3 + 4 * M + N * K + 4 * N + 2 * M * N)
+        config = {"workload": f"channel-wise W8A8 linear, DeepSeek-R1 MoE expert down-proj "
+                              f"X[{M},{K}] W[{N},{K}] bf16 out; step = per-token act quant + INT8 GEMM",
+                  "M": M, "N": N, "K": K, "global_batch": M * world, "seq_len": 1,
+                  "parallelism": f"dp{world}", "l2": f"{R} rotating input/output copies (> 2x L2 per cycle)"}
+    elif name == "w8a8_block":
+        N, K = (18432, 7168) if args.proj == "up" else (7168, 18432)
+        M = args.M or 4096
+        KB, ld = K // 128, (M + 3) // 4 * 4
+        R = _rotations(M * K * 3 + 4 * KB * ld + N * K + 2 * M * N)
+        config = {"workload": f"block-wise W8A8 linear, DeepSeek-R1 dense MLP {args.proj}-proj X[{M},{K}] "
+                              f"W[{N},{K}] bf16 out; step = per-token-group act quant + INT8 GEMM",
+                  "M": M, "N": N, "K": K, "global_batch": M * world, "seq_len": 1,
+                  "parallelism": f"dp{world}", "l2": f"{R} rotating input/output copies (> 2x L2 per cycle)"}
+    elif name == "requant":
+        M, N, K, R = 0, 18432, 7168, 2
+        config = {"workload": f"offline FP8-E4M3 [{N},{K}] (128x128 fp32 scales) -> BF16 -> INT8 128x128 block requant",
+                  "N": N, "K": K, "parallelism": f"dp{world}", "l2": "2 rotating copies of 264 MB"}
+    elif name == "w8a16":
+        M = args.M or 16
+        N, K = (12288, 4096) if args.proj == "up" else (4096, 12288)
+        R = _rotations(N * K + 2 * N * (K // 128) + 2 * M * K + 2 * M * N)
+        config = {"workload": f"W8A16 group-128 decode GEMM, Qwen3-8B linear X fp16[{M},{K}] W int8[{N},{K}]",
+                  "M": M, "N": N, "K": K, "global_batch": M * world, "parallelism": f"dp{world}",
+                  "l2": f"{R} rotating copies (> 2x L2 per cycle)"}
+    else:
+        raise ValueError(name)
+    return {"M": M, "N": N, "K": K, "R": R, "config": config}
+
+
 class ChannelW8A8(Workload):
     name = "w8a8_channel"
 
@@ -152,11 +188,7 @@ class ChannelW8A8(Workload):
         self.dom_bytes = M * K + 4 * M + N * K + 4 * N + 2 * M * N
         self.h2d_bytes = M * K * 2
         self.d2h_bytes = M * N * 2
-        self.config = {"workload": f"channel-wise W8A8 linear, DeepSeek-R1 MoE expert down-proj "
-                                   f"X[{M},{K}] W[{N},{K}] bf16 out; step = per-token act quant + INT8 GEMM",
-                       "M": M, "N": N, "K": K, "global_batch": M * args.world, "seq_len": 1,
-                       "parallelism": f"dp{args.world}",
-                       "l2": f"{self.R} rotating input/output copies (> 2x L2 per cycle)"}
+        self.config = describe(self.name, args)["config"]
 
     def launch(self, i, k, stream):
         b = self.bufs[i % self.R]
@@ -235,11 +267,7 @@ class BlockW8A8(Workload):
         self.dom_bytes = M * K + 4 * M * KB + N * K + 4 * ((N + 127) // 128) * KB + 2 * M * N
         self.h2d_bytes = M * K * 2
         self.d2h_bytes = M * N * 2
-        self.config = {"workload": f"block-wise W8A8 linear, DeepSeek-R1 dense MLP {proj}-proj X[{M},{K}] "
-                                   f"W[{N},{K}] bf16 out; step = per-token-group act quant + INT8 GEMM",
-                       "M": M, "N": N, "K": K, "global_batch": M * args.world, "seq_len": 1,
-                       "parallelism": f"dp{args.world}",
-                       "l2": f"{self.R} rotating input/output copies (> 2x L2 per cycle)"}
+        self.config = describe(self.name, args)["config"]
 
     def launch(self, i, k, stream):
         b = self.bufs[i % self.R]
@@ -300,8 +328,7 @@ class Requant(Workload):
         self.dom_bytes = nbytes
         self.h2d_bytes = N * K
         self.d2h_bytes = N * K
-        self.config = {"workload": f"offline FP8-E4M3 [{N},{K}] (128x128 fp32 scales) -> BF16 -> INT8 128x128 block requant",
-                       "N": N, "K": K, "parallelism": f"dp{args.world}", "l2": "2 rotating copies of 264 MB"}
+        self.config = describe(self.name, args)["config"]
 
     def launch(self, i, k, stream):
         b = self.bufs[i % self.R]
@@ -357,9 +384,7 @@ class W8A16(Workload):
         self.dom_bytes = per_copy
         self.h2d_bytes = 2 * M * K
         self.d2h_bytes = 2 * M * N
-        self.config = {"workload": f"W8A16 group-128 decode GEMM, Qwen3-8B linear X fp16[{M},{K}] W int8[{N},{K}]",
-                       "M": M, "N": N, "K": K, "global_batch": M * args.world, "parallelism": f"dp{args.world}",
-                       "l2": f"{self.R} rotating copies (> 2x L2 per cycle)"}
+        self.config = describe(self.name, args)["config"]
 
     def launch(self, i, k, stream):
         b = self.bufs[i % self.R]
@@ -571,31 +596,15 @@ def run_reference(args):
         return
     args.world = world
 
-    class _Stub:
-        pass
     cls = WORKLOADS[args.workload]
     wl = cls.__new__(cls)
     wl.args = args
-    # shapes only (no device buffers): reuse the constructors' sizes without touching CUDA
-    if args.workload == "w8a8_channel":
-        wl.M, wl.N, wl.K = args.M or 4096, 7168, 2048
-        wl.unit = "TOPS"
-        cfg = {"workload": f"channel-wise W8A8 linear, DeepSeek-R1 MoE expert down-proj X[{wl.M},2048] W[7168,2048]"}
-    elif args.workload == "w8a8_block":
-        wl.N, wl.K = (18432, 7168) if args.proj == "up" else (7168, 18432)
-        wl.M = args.M or 4096
-        wl.unit = "TOPS"
-        cfg = {"workload": f"block-wise W8A8 linear, DeepSeek-R1 dense MLP {args.proj}-proj"}
-    elif args.workload == "requant":
-        wl.N, wl.K = 18432, 7168
-        wl.unit = "GB/s"
-        cfg = {"workload": "offline FP8 -> BF16 -> INT8 block requant [18432,7168]"}
-    else:
-        wl.M = args.M or 16
-        wl.N, wl.K = (12288, 4096) if args.proj == "up" else (4096, 12288)
-        wl.unit = "GB/s"
+    # shapes only (no device buffers); the config is the GPU arm's
+    d = describe(args.workload, args)
+    wl.M, wl.N, wl.K = d["M"], d["N"], d["K"]
+    cfg = d["config"]
+    if args.workload == "w8a16":
         wl.units_per_step = (wl.N * wl.K + 2 * wl.N * (wl.K // 128) + 2 * wl.M * wl.K + 2 * wl.M * wl.N) / 1e9
-        cfg = {"workload": f"W8A16 decode M={wl.M} N={wl.N} K={wl.K}"}
     budget = max(0.5, min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         wl.oracle_sample(budget)

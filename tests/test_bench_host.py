@@ -1,0 +1,59 @@
+"""Host-side logic of bench.py that needs no GPU: the reference arm (the oracle on the host cores)
+prints one JSON line with the GPU arm's config, metric and unit; the traffic table is keyed by the
+workload's shape."""
+import io
+import json
+import types
+from contextlib import redirect_stdout
+
+import pytest
+
+import bench
+
+
+def _args(workload, **kw):
+    a = types.SimpleNamespace(workload=workload, M=0, proj="up", steps=1, warmup=0, cpu_budget=0.2,
+                              gpus=1, world=1)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("workload,kw", [("w8a8_channel", {"M": 16}), ("w8a16", {"M": 4, "proj": "down"}),
+                                         ("w8a8_block", {"M": 1, "proj": "down"})])
+def test_reference_line_matches_gpu_arm_config(workload, kw):
+    args = _args(workload, **kw)
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.run_reference(args)
+    line = json.loads(buf.getvalue().strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC
+    assert line["config"] == bench.describe(workload, args)["config"]
+    assert line["unit"] == bench.WORKLOADS[workload].unit
+    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_describe_shapes():
+    d = bench.describe("w8a8_block", _args("w8a8_block", M=16384))
+    assert (d["M"], d["N"], d["K"]) == (16384, 18432, 7168) and d["R"] >= 1
+    d = bench.describe("w8a8_block", _args("w8a8_block", proj="down"))
+    assert (d["M"], d["N"], d["K"]) == (4096, 7168, 18432)
+    d = bench.describe("w8a16", _args("w8a16"))
+    assert (d["M"], d["N"], d["K"]) == (16, 12288, 4096)
+    assert bench.describe("w8a8_channel", _args("w8a8_channel", world=4))["config"]["global_batch"] == 4 * 4096
+
+
+def test_measured_traffic_lookup():
+    traffic, src = bench.measured_traffic("w8a8_channel", {"M": 4096, "N": 7168, "K": 2048})
+    assert traffic and src.endswith(".md")
+    assert bench.measured_traffic("w8a8_channel", {"M": 7, "N": 7168, "K": 2048}) == (None, None)
+
+
+def test_traffic_sources_exist():
+    import os
+    root = os.path.dirname(os.path.abspath(bench.__file__))
+    for key, (traffic, src) in bench.MEASURED_TRAFFIC.items():
+        assert traffic > 0, key
+        assert os.path.exists(os.path.join(root, "profiles", src)), (key, src)
