@@ -39,7 +39,7 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_max_time_and_shards():
     world = 2
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:   # no fork of a multi-threaded test process
         out = m.dict()
         mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
