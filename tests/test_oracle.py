@@ -87,6 +87,25 @@ def test_fp8_dequant_vs_torch_route():
     assert np.array_equal(got, ref)
 
 
+def test_fp8_block_absmax_is_the_largest_code_dequantized():
+    """bf16(fp32(e) * sf) is monotone in |e| for sf > 0, and |e| is monotone in the code's low 7 bits,
+    so a block's BF16 absmax is the dequantization of its largest code: checked on every block of a
+    checkpoint, including all-zero and single-code blocks."""
+    w8, sf = synth.fp8_checkpoint(384, 512, seed=16)
+    w8 = w8.copy()
+    w8[:128, :128] = 0                      # all-zero block
+    w8[128:256, 128:256] = 0x80 | 0x35      # one negative code everywhere
+    bf = O.dequant_fp8_block_to_bf16(w8, sf)
+    mag = np.abs(O.bf16_to_f32(bf))
+    for i in range(3):
+        for j in range(4):
+            blk = (slice(i * 128, (i + 1) * 128), slice(j * 128, (j + 1) * 128))
+            code = int((w8[blk] & 0x7F).max())
+            one = np.array([[code]], dtype=np.uint8)
+            expect = float(np.abs(O.bf16_to_f32(O.dequant_fp8_block_to_bf16(one, sf[i:i + 1, j:j + 1])))[0, 0])
+            assert float(mag[blk].max()) == expect
+
+
 def test_requant_is_dequant_then_block_quant():
     w8, sf = synth.fp8_checkpoint(256, 256, seed=15)
     wq, sw = O.requant_fp8_to_int8_block(w8, sf)
