@@ -22,8 +22,17 @@ enum WaitSite : unsigned {
 };
 
 // A wait gives up after this many nanoseconds of %globaltimer (no kernel here legitimately
-// waits anywhere near this long on one barrier phase).
+// waits anywhere near this long on one barrier phase).  g_wait_limit_ns holds the limit of the
+// pipeline waits and may be lowered for a test (i8q_test_set_wait_limit_ns); the drain waits,
+// which let copies and MMAs already in flight finish before a CTA exits, always use the default.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
+__device__ unsigned long long g_wait_limit_ns = kWaitTimeoutNs;
+
+// Test aid, normally 0.  When set (i8q_test_skip_accumulator_signal), the first CTA of the
+// decode-size channel-wise W8A8 GEMM that reads it clears it and withholds its accumulator-ready
+// signal once, so that its epilogue's bounded wait expires: the kernel then returns early and
+// i8q_status_check() reports I8Q_ERR_TIMEOUT.  Nothing else in flight depends on that signal.
+__device__ unsigned int g_test_skip_acc_signal;
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
@@ -79,11 +88,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
                                           volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = globaltimer_ns();
+  const unsigned long long limit =
+      site == SITE_DRAIN ? (unsigned long long)kWaitTimeoutNs
+                         : *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (abort_flag && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit) {
         raise_error(site);
         if (abort_flag) *abort_flag = 1;
         return false;

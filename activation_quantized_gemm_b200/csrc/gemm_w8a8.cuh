@@ -185,20 +185,30 @@ __device__ __forceinline__ void store_row8(void* y, bool f32out, int64_t off, co
 // columns nc .. nc + W - 1 (W = 16 or 32) of row m_base + l as bf16 pairs.  The 32 rows go through
 // a 32 x 80-byte staging slab in shared memory (80-byte rows: conflict-free for row-wise writes and
 // column-wise reads), then each store instruction writes 8 rows x 64 contiguous bytes instead of
-// 16 bytes of 32 different rows (half-filled sectors).
+// 16 bytes of 32 different rows (half-filled sectors).  When N % 8 != 0 the rows of y are not
+// 16-byte aligned: every element is then stored on its own (lane = column), masked at N.
 __device__ __forceinline__ void store_rows_bf16(uint8_t* stg, int lane, const uint32_t (&p)[16], int W, uint16_t* y,
-                                                int N, int m_base, int M, int nc) {
+                                                int N, int m_base, int M, int nc, bool nvec) {
   uint4* srow = reinterpret_cast<uint4*>(stg + lane * 80);
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     if (q * 8 < W) srow[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
   __syncwarp();
+  if (nvec) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = i * 8 + (lane & 7), c = lane >> 3;
-    const int m = m_base + r, n = nc + c * 8;
-    if (c * 8 < W && m < M && n < N)
-      *reinterpret_cast<uint4*>(y + (int64_t)m * N + n) = *reinterpret_cast<const uint4*>(stg + r * 80 + c * 16);
+    for (int i = 0; i < 4; ++i) {
+      const int r = i * 8 + (lane & 7), c = lane >> 3;
+      const int m = m_base + r, n = nc + c * 8;
+      if (c * 8 < W && m < M && n < N)
+        *reinterpret_cast<uint4*>(y + (int64_t)m * N + n) = *reinterpret_cast<const uint4*>(stg + r * 80 + c * 16);
+    }
+  } else {
+    const int n = nc + lane;
+#pragma unroll 4
+    for (int r = 0; r < 32; ++r) {
+      const int m = m_base + r;
+      if (lane < W && m < M && n < N) y[(int64_t)m * N + n] = reinterpret_cast<const uint16_t*>(stg + r * 80)[lane];
+    }
   }
   __syncwarp();
 }
@@ -235,6 +245,7 @@ __global__ void __launch_bounds__(384, 1)
   const int M = args.M, N = args.N, K = args.K;
   const int Mt = (M + GEMM_BM - 1) / GEMM_BM, Nt = (N + BN - 1) / BN, KB = K / GEMM_BK;
   const int num_tiles = Mt * Nt;
+  const bool nvec = (N & 7) == 0;   // rows of y, sw and the debug outputs allow vector accesses
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -389,12 +400,19 @@ __global__ void __launch_bounds__(384, 1)
           for (int g = 0; g < 4; ++g) {
             const int n = nc + g * 8;
             if (g * 8 < W) {
-              float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
-              if (n < N) {
-                w0 = __ldg(reinterpret_cast<const float4*>(args.sw + n));
-                w1 = __ldg(reinterpret_cast<const float4*>(args.sw + n + 4));
+              float ws[8];
+              if (nvec) {
+                float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
+                if (n < N) {
+                  w0 = __ldg(reinterpret_cast<const float4*>(args.sw + n));
+                  w1 = __ldg(reinterpret_cast<const float4*>(args.sw + n + 4));
+                }
+                ws[0] = w0.x; ws[1] = w0.y; ws[2] = w0.z; ws[3] = w0.w;
+                ws[4] = w1.x; ws[5] = w1.y; ws[6] = w1.z; ws[7] = w1.w;
+              } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ws[j] = n + j < N ? __ldg(args.sw + n + j) : 0.f;
               }
-              const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
               float v[8];
 #pragma unroll
               for (int j = 0; j < 8; ++j) v[j] = __int2float_rn((int)r[g * 8 + j]) * (sxm * ws[j]);
@@ -402,14 +420,20 @@ __global__ void __launch_bounds__(384, 1)
               for (int j = 0; j < 4; ++j) pk[g * 4 + j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
               if constexpr (DEBUG) {
                 if (row_ok && n < N) {
-                  int4* dp = reinterpret_cast<int4*>(args.dbg + (int64_t)m * N + n);
-                  dp[0] = make_int4(r[g * 8 + 0], r[g * 8 + 1], r[g * 8 + 2], r[g * 8 + 3]);
-                  dp[1] = make_int4(r[g * 8 + 4], r[g * 8 + 5], r[g * 8 + 6], r[g * 8 + 7]);
+                  if (nvec) {
+                    int4* dp = reinterpret_cast<int4*>(args.dbg + (int64_t)m * N + n);
+                    dp[0] = make_int4(r[g * 8 + 0], r[g * 8 + 1], r[g * 8 + 2], r[g * 8 + 3]);
+                    dp[1] = make_int4(r[g * 8 + 4], r[g * 8 + 5], r[g * 8 + 6], r[g * 8 + 7]);
+                  } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                      if (n + j < N) args.dbg[(int64_t)m * N + n + j] = (int32_t)r[g * 8 + j];
+                  }
                 }
               }
             }
           }
-          store_rows_bf16(stg, lane, pk, W, reinterpret_cast<uint16_t*>(args.y), N, m - lane, M, nc);
+          store_rows_bf16(stg, lane, pk, W, reinterpret_cast<uint16_t*>(args.y), N, m - lane, M, nc, nvec);
         };
 #pragma unroll 1
         for (int c = 0; c < HALF / 32; ++c) {
@@ -494,7 +518,13 @@ __global__ void __launch_bounds__(384, 1)
                   v[2 * j] = sum[g * 4 + j].x;
                   v[2 * j + 1] = sum[g * 4 + j].y;
                 }
-                store_row8(args.y, true, (int64_t)m * N + n, v);
+                if (nvec) {
+                  store_row8(args.y, true, (int64_t)m * N + n, v);
+                } else {
+#pragma unroll
+                  for (int j = 0; j < 8; ++j)
+                    if (n + j < N) reinterpret_cast<float*>(args.y)[(int64_t)m * N + n + j] = v[j];
+                }
               }
             }
           }
@@ -504,7 +534,7 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(sum[c * 16 + j].x, sum[c * 16 + j].y);
-            store_rows_bf16(stg, lane, pk, 32, reinterpret_cast<uint16_t*>(args.y), N, m - lane, M, n0 + c * 32);
+            store_rows_bf16(stg, lane, pk, 32, reinterpret_cast<uint16_t*>(args.y), N, m - lane, M, n0 + c * 32, nvec);
           }
         }
       }

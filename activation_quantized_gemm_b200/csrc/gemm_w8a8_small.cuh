@@ -180,7 +180,12 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS,
         tc_commit(&empty[s]);
         if (BLOCKWISE) tc_commit(&tfull[b]);
       }
-      if (!BLOCKWISE) tc_commit(&tfull[0]);
+      if (!BLOCKWISE) {
+        // test aid (see g_test_skip_acc_signal): withhold this signal once, when armed
+        const bool skip = *reinterpret_cast<volatile unsigned*>(&g_test_skip_acc_signal) != 0 &&
+                          atomicExch(&g_test_skip_acc_signal, 0u) != 0;
+        if (!skip) tc_commit(&tfull[0]);
+      }
       tc_commit(done);
       mbar_wait(done, 0, SITE_DRAIN, nullptr);
     }

@@ -156,9 +156,26 @@ static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t
 
 static inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Dynamic shared memory above 48 KB must be opted into per kernel, and the attribute belongs to
+// the current device: it is set once per (kernel, device).
+static std::mutex g_smem_mu;
+static const void* g_smem_kern[256];
+static int g_smem_dev[256];
+static int g_smem_n = 0;
+
 template <typename Kern>
-static i8q_status set_smem(Kern k, int bytes) {
+static i8q_status ensure_smem(Kern k, int bytes) {
+  int dev = 0;
+  I8Q_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_smem_mu);
+  for (int i = 0; i < g_smem_n; ++i)
+    if (g_smem_kern[i] == (const void*)k && g_smem_dev[i] == dev) return I8Q_OK;
   I8Q_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  if (g_smem_n < 256) {
+    g_smem_kern[g_smem_n] = (const void*)k;
+    g_smem_dev[g_smem_n] = dev;
+    ++g_smem_n;
+  }
   return I8Q_OK;
 }
 
@@ -227,9 +244,7 @@ static i8q_status launch_w8a16_mp(const uint16_t* x, const int8_t* wq, const uin
                                   uint16_t* y, int sms, cudaStream_t stream) {
   using C = W8A16Cfg<MP>;
   auto kern = k_gemm_w8a16<MP>;
-  static std::once_flag once;
-  static i8q_status attr = I8Q_OK;
-  std::call_once(once, [&] { attr = set_smem(kern, C::SMEM_BYTES); });
+  const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
   if (attr) return attr;
   CUtensorMap tw, tx;
   i8q_status st = make_tmap_2d(&tw, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, W8A16_BN, 128,
@@ -269,7 +284,7 @@ static i8q_status launch_w8a16(const uint16_t* x, const int8_t* wq, const uint16
 static i8q_status gemm_w8a8_common_checks(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
                                           int64_t M, int64_t N, int64_t K, const void* y, const void* dbg) {
   I8Q_REQUIRE(M >= 0 && N >= 0 && K >= 0 && M < kMaxDim && N < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
-  I8Q_REQUIRE(K % 128 == 0 && N % 8 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(K % 128 == 0, I8Q_ERR_SHAPE);
   I8Q_REQUIRE(127LL * 127LL * K < (1LL << 31), I8Q_ERR_SHAPE);
   if (M == 0 || N == 0) return I8Q_OK;
   I8Q_REQUIRE(y, I8Q_ERR_NULL);
@@ -284,9 +299,7 @@ template <int BN, bool BLOCKWISE, bool F32, bool DBG>
 static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms, cudaStream_t s) {
   using C = W8A8Cfg<BN>;
   auto kern = k_gemm_w8a8<BN, BLOCKWISE, F32, DBG>;
-  static std::once_flag once;
-  static i8q_status attr = I8Q_OK;
-  std::call_once(once, [&] { attr = set_smem(kern, C::SMEM_BYTES); });
+  const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
   if (attr) return attr;
   CUtensorMap ta, tb;
   i8q_status st = make_tmap_2d(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, a.K, 128, GEMM_BK,
@@ -323,9 +336,7 @@ static i8q_status launch_w8a8_small_mp(const int8_t* xq, const int8_t* wq, const
   constexpr int CPS = MP <= 64 ? 2 : 1;   // 128 tokens: one CTA per SM (TMEM and registers)
   using C = W8A8SmallCfg<MP, BLOCKWISE, CPS>;
   auto kern = k_gemm_w8a8_small<MP, BLOCKWISE, CPS, F32, DBG>;
-  static std::once_flag once;
-  static i8q_status attr = I8Q_OK;
-  std::call_once(once, [&] { attr = set_smem(kern, C::SMEM_BYTES); });
+  const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
   if (attr) return attr;
   CUtensorMap tw, tx;
   i8q_status st = make_tmap_2d(&tw, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, a.K, 128, 128,
@@ -426,6 +437,19 @@ i8q_status i8q_status_check(void* stream) {
   return I8Q_OK;
 }
 
+// ---------------------------------------------------------------- test aids ------------------
+i8q_status i8q_test_set_wait_limit_ns(uint64_t ns) {
+  unsigned long long v = ns ? (unsigned long long)ns : kWaitTimeoutNs;
+  I8Q_CUDA(cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)));
+  return I8Q_OK;
+}
+
+i8q_status i8q_test_skip_accumulator_signal(int armed) {
+  unsigned int v = armed ? 1u : 0u;
+  I8Q_CUDA(cudaMemcpyToSymbol(g_test_skip_acc_signal, &v, sizeof(v)));
+  return I8Q_OK;
+}
+
 // ---------------------------------------------------------------- a1 -------------------------
 i8q_status i8q_quant_act_token_group(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int8_t* xq, float* sx,
                                      int64_t ld_sx, void* stream) {
@@ -455,7 +479,7 @@ i8q_status i8q_quant_act_token_group(const uint16_t* x, int64_t M, int64_t K, in
 i8q_status i8q_quant_act_token(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int8_t* xq, float* sx,
                                void* stream) {
   I8Q_REQUIRE(M >= 0 && K >= 0 && M < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
-  I8Q_REQUIRE(K % 16 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(K % 8 == 0, I8Q_ERR_SHAPE);   // rows move as 16-byte bf16 / 8-byte int8 vectors
   if (M == 0) return I8Q_OK;
   I8Q_REQUIRE(x && xq && sx, I8Q_ERR_NULL);
   I8Q_REQUIRE(ldx >= K && ldx % 8 == 0, I8Q_ERR_SHAPE);
@@ -584,7 +608,7 @@ i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx,
 i8q_status i8q_gemm_w8a16_group(const uint16_t* x, const int8_t* wq, const uint16_t* s, int64_t M, int64_t N,
                                 int64_t K, uint16_t* y, void* stream) {
   I8Q_REQUIRE(M >= 0 && N >= 0 && K >= 0 && N < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
-  I8Q_REQUIRE(M <= W8A16_MAX_M && K % 128 == 0 && N % 8 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(M <= W8A16_MAX_M && K % 128 == 0, I8Q_ERR_SHAPE);
   if (M == 0 || N == 0) return I8Q_OK;
   I8Q_REQUIRE(y, I8Q_ERR_NULL);
   I8Q_REQUIRE(aligned16(y), I8Q_ERR_ALIGN);

@@ -48,6 +48,8 @@ _SIGS = {
     "i8q_gemm_w8a8_channel": [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P],
     "i8q_gemm_w8a16_group": [_P, _P, _P, _I, _I, _I, _P, _P],
     "i8q_status_check": [_P],
+    "i8q_test_set_wait_limit_ns": [ctypes.c_uint64],
+    "i8q_test_skip_accumulator_signal": [ctypes.c_int],
     "i8q_status_string": [ctypes.c_int],
     "i8q_last_error_string": [],
     "i8q_version": [],
@@ -169,6 +171,16 @@ def i8q_gemm_w8a16_group(x, wq, s, y, stream=None) -> None:
 def i8q_status_check(stream=None) -> None:
     """Synchronize the stream; raise I8QError(I8Q_ERR_TIMEOUT) if a bounded device wait expired."""
     _call("i8q_status_check", _stream(stream))
+
+
+def i8q_test_set_wait_limit_ns(ns: int) -> None:
+    """Test aid: limit of the pipeline waits on the current device in ns (0 = the 2 s default)."""
+    _call("i8q_test_set_wait_limit_ns", int(ns))
+
+
+def i8q_test_skip_accumulator_signal(armed: bool = True) -> None:
+    """Test aid: the next decode-size channel-wise W8A8 GEMM withholds one accumulator signal."""
+    _call("i8q_test_skip_accumulator_signal", 1 if armed else 0)
 
 
 def i8q_status_string(status: int) -> str:

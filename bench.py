@@ -1,25 +1,30 @@
 #!/usr/bin/env python
 """Benchmark of the symmetric INT8 activation-quantized linear layer on B200.
 
-Default workload (one "step" = the whole hot path of one channel-wise W8A8 linear layer):
-DeepSeek-R1 MoE expert down-projection shape, X bf16 [M=4096, K=2048] (~N(0,1), 0.1% of
-entries x50), W [N=7168, K=2048] (~N(0,0.02)) quantized per output channel offline; per step:
-online per-token activation quantization (i8q_quant_act_token) + channel-wise INT8 GEMM with
-bf16 output (i8q_gemm_w8a8_channel).  Other workloads (--workload) cover the block-wise layer,
-the offline requantization and the W8A16 decode GEMM.
+Default workload (one "step" = the whole hot path of one block-wise W8A8 linear layer, the pages'
+primary scheme): DeepSeek-R1 dense-MLP up-projection, X bf16 [M=16384, K=7168] (~N(0,1), 0.1% of
+entries x50), W [N=18432, K=7168] (~N(0,0.02)) quantized in 128x128 blocks offline; per step:
+online per-token-group activation quantization (i8q_quant_act_token_group) + block-wise INT8 GEMM
+with per-slab dequantization and bf16 output (i8q_gemm_w8a8_block).  `value` is TOPS of that step.
+
+The same JSON line carries `sub_results`: the other kernels of the metric ("quant-kernel GB/s & %
+of HBM peak", decode GEMMs as GB/s), each timed in this run on its own configured shape: the
+per-token-group quantizer of the default step, the channel-wise layer (MoE expert down-proj,
+M = 4096 and M = 16), block-wise decode (M = 16, up and down), the offline FP8 requant and the
+W8A16 decode GEMM (Qwen3-8B shapes, M = 16).  Other workloads are available with --workload.
 
 Timing: W warm-up steps, then K steps back to back between CUDA events on the launching stream,
 cycling through enough independent copies of every input and output that the working set of a
 cycle exceeds twice the 126 MB L2 (no step reads what the previous one left in L2).  The timed
 region holds only the steps' kernels, so a GEMM may overlap its start-up with the kernel before
 it (programmatic dependent launch).  A second pass of K steps brackets every kernel with its own
-events, which gives each kernel's average launch duration (the roofline figure).  With torchrun
-(N > 1) every rank runs the same per-GPU workload on its own tokens (data-parallel, weights
-replicated, no collective on the data path): weak scaling, value = all ranks' work /
-max-over-ranks time.
+events, which gives each kernel's average launch duration (the roofline figure).  With N > 1
+(`--gpus N` spawns one process per GPU itself, or torchrun launches them) every rank runs the same
+per-GPU workload on its own tokens (data-parallel, weights replicated, no collective on the data
+path): weak scaling, value = all ranks' work / max-over-ranks time.
 
-`--impl reference` times the CPU oracle (tests' reference implementation) on a bounded sample
-of the same workload instead.
+`--impl reference` times the CPU oracle (the plain C++ oracle the tests compare with, OpenMP over
+all host cores) on a bounded sample of the same workload instead.
 """
 from __future__ import annotations
 
@@ -55,10 +60,6 @@ def load_peaks():
 # bench's own command (profiles/<file>.md), keyed by (workload, M, N, K).  A kernel change
 # invalidates its entry: it must then be re-measured or removed (the line reports null).
 MEASURED_TRAFFIC = {
-    ("w8a8_channel", 4096, 7168, 2048): (36.13e6, "w8a8_channel_m4096.md"),
-    ("w8a8_channel", 16, 7168, 2048): (14.77e6, "w8a8_small_channel_m16.md"),
-    ("w8a8_block", 16384, 18432, 7168): (1824.7e6, "w8a8_block_up_m16384.md"),
-    ("w8a8_block", 16, 18432, 7168): (138.08e6, "w8a8_small_block_up_m16.md"),
     ("requant", 0, 18432, 7168): (217.65e6, "requant_fp8_block_n18432_k7168.md"),
     ("w8a16", 16, 12288, 4096): (51.30e6, "w8a16_m16_n12288_k4096.md"),
     ("w8a16", 16, 4096, 12288): (51.55e6, "w8a16_m16_n4096_k12288.md"),
@@ -114,6 +115,12 @@ def _rotations(bytes_per_copy: int) -> int:
     return max(1, min(16, -(-2 * L2_BYTES // max(1, bytes_per_copy)) + 1))
 
 
+def _scale_rows(run, lo: int, hi: int, budget_s: float) -> int:
+    """Rows of an oracle sample that take about `budget_s` seconds: time `lo` rows, then scale."""
+    dt = max(run(lo), 1e-4)
+    return int(max(lo, min(hi, lo * budget_s / dt)))
+
+
 def describe(name: str, args) -> dict:
     """Shapes, rotation count and the JSON `config` of a workload, from the arguments alone (no
     device buffers): the GPU arm and the reference arm report the same config."""
@@ -127,7 +134,7 @@ def describe(name: str, args) -> dict:
                   "parallelism": f"dp{world}", "l2": f"{R} rotating input/output copies (> 2x L2 per cycle)"}
     elif name == "w8a8_block":
         N, K = (18432, 7168) if args.proj == "up" else (7168, 18432)
-        M = args.M or 4096
+        M = args.M or 16384
         KB, ld = K // 128, (M + 3) // 4 * 4
         R = _rotations(M * K * 3 + 4 * KB * ld + N * K + 2 * M * N)
         config = {"workload": f"block-wise W8A8 linear, DeepSeek-R1 dense MLP {args.proj}-proj X[{M},{K}] "
@@ -205,23 +212,28 @@ class ChannelW8A8(Workload):
         self.y_host.copy_(b["y"], non_blocking=True)
 
     def oracle_sample(self, budget_s):
-        """Oracle on a row subset of the same workload; returns (units, seconds, description)."""
-        import oracle as O
+        """The C++ oracle on a row subset of the same workload; returns (units, seconds, description)."""
+        from oracle import ref_cpp as O
         from activation_quantized_gemm_b200 import synth
         w = synth.weight_bf16(self.N, self.K, seed=1)
         wq, sw = O.quant_act_token(w)                              # offline, not timed
-        rows = 8
-        x = synth.activation_bf16(self.M, self.K, seed=1, outlier_p=0.001, outlier_mult=50.0)
-        t0 = time.perf_counter()
-        xq, sx = O.quant_act_token(x[:rows])
-        O.gemm_w8a8_channel(xq, sx, wq, sw)
-        dt = time.perf_counter() - t0
-        rows = int(max(8, min(self.M, rows * budget_s / max(dt, 1e-3))))
-        t0 = time.perf_counter()
-        xq, sx = O.quant_act_token(x[:rows])
-        O.gemm_w8a8_channel(xq, sx, wq, sw)
-        dt = time.perf_counter() - t0
+        x = synth.activation_bf16(min(self.M, 1024), self.K, seed=1, outlier_p=0.001, outlier_mult=50.0)
+
+        def run(rows):
+            t0 = time.perf_counter()
+            xq, sx = O.quant_act_token(x[:rows])
+            O.gemm_w8a8_channel(xq, sx, wq, sw)
+            return time.perf_counter() - t0
+        rows = _scale_rows(run, 4, x.shape[0], budget_s)
+        dt = run(rows)
         return 2.0 * rows * self.N * self.K / 1e12, dt, f"{rows} of {self.M} token rows (quant + GEMM), N={self.N}, K={self.K}"
+
+    def sub_results(self):
+        """Per-kernel figures of this workload: the per-token quantizer and the GEMM."""
+        M, N, K = self.M, self.N, self.K
+        return [("quant_act_token", f"a2 per-token act quant [{M},{K}]", "hbm", 3 * M * K + 4 * M),
+                ("gemm_w8a8_channel", f"a5 channel-wise GEMM M={M} N={N} K={K}",
+                 self.dom_bound, self.dom_units * 1e12 if self.dom_bound == "tensor" else self.dom_bytes)]
 
 
 class BlockW8A8(Workload):
@@ -234,7 +246,7 @@ class BlockW8A8(Workload):
         self.q = i8q
         proj = args.proj
         N, K = (18432, 7168) if proj == "up" else (7168, 18432)
-        M = args.M or 4096
+        M = args.M or 16384
         self.M, self.N, self.K = M, N, K
         x = synth.activation_bf16(M, K, seed=shard_seed(2, rank), outlier_p=0.001, outlier_mult=50.0)
         w = synth.weight_bf16(N, K, seed=2)
@@ -284,17 +296,28 @@ class BlockW8A8(Workload):
         self.y_host.copy_(b["y"], non_blocking=True)
 
     def oracle_sample(self, budget_s):
-        import oracle as O
+        from oracle import ref_cpp as O
         from activation_quantized_gemm_b200 import synth
         w = synth.weight_bf16(self.N, self.K, seed=2)
-        wq, sw = O.quant_weight_block(w)
-        x = synth.activation_bf16(8, self.K, seed=2, outlier_p=0.001, outlier_mult=50.0)
-        rows = 4
-        t0 = time.perf_counter()
-        xq, sx = O.quant_act_token_group(x[:rows])
-        O.gemm_w8a8_block(xq, sx, wq, sw)
-        dt = time.perf_counter() - t0
+        wq, sw = O.quant_weight_block(w)                           # offline, not timed
+        x = synth.activation_bf16(min(self.M, 256), self.K, seed=2, outlier_p=0.001, outlier_mult=50.0)
+
+        def run(rows):
+            t0 = time.perf_counter()
+            xq, sx = O.quant_act_token_group(x[:rows])
+            O.gemm_w8a8_block(xq, sx, wq, sw)
+            return time.perf_counter() - t0
+        rows = _scale_rows(run, 1, x.shape[0], budget_s)
+        dt = run(rows)
         return 2.0 * rows * self.N * self.K / 1e12, dt, f"{rows} of {self.M} token rows (quant + GEMM), N={self.N}, K={self.K}"
+
+    def sub_results(self):
+        M, N, K = self.M, self.N, self.K
+        KB = K // 128
+        return [("quant_act_token_group", f"a1 per-token-group act quant [{M},{K}]", "hbm",
+                 3 * M * K + 4 * M * KB),
+                ("gemm_w8a8_block", f"a4 block-wise GEMM {self.args.proj}-proj M={M} N={N} K={K}",
+                 self.dom_bound, self.dom_units * 1e12 if self.dom_bound == "tensor" else self.dom_bytes)]
 
 
 class Requant(Workload):
@@ -341,14 +364,23 @@ class Requant(Workload):
         self.wq_host.copy_(b["wq"], non_blocking=True)
 
     def oracle_sample(self, budget_s):
-        import oracle as O
+        from oracle import ref_cpp as O
         from activation_quantized_gemm_b200 import synth
-        rows = 1024
-        w8, sf = synth.fp8_checkpoint(rows, self.K, seed=3)
-        t0 = time.perf_counter()
-        O.requant_fp8_to_int8_block(w8, sf)
-        dt = time.perf_counter() - t0
-        return (rows * self.K * 2 + 8 * sf.size) / 1e9, dt, f"{rows} of {self.N} weight rows"
+        w8, sf = synth.fp8_checkpoint(self.N, self.K, seed=3)
+
+        def run(rows):
+            rows128 = -(-rows // 128) * 128
+            t0 = time.perf_counter()
+            O.requant_fp8_to_int8_block(w8[:rows128], sf[:rows128 // 128])
+            return time.perf_counter() - t0
+        rows = _scale_rows(run, 128, self.N, budget_s)
+        rows = -(-rows // 128) * 128
+        dt = run(rows)
+        return (rows * self.K * 2 + 8 * (rows // 128) * (self.K // 128)) / 1e9, dt, f"{rows} of {self.N} weight rows"
+
+    def sub_results(self):
+        return [("requant_fp8_to_int8_block", f"a3 FP8 -> BF16 -> INT8 block requant [{self.N},{self.K}]", "hbm",
+                 self.dom_bytes)]
 
 
 class W8A16(Workload):
@@ -397,14 +429,22 @@ class W8A16(Workload):
         self.y_host.copy_(b["y"], non_blocking=True)
 
     def oracle_sample(self, budget_s):
-        import oracle as O
+        from oracle import ref_cpp as O
         from activation_quantized_gemm_b200 import synth
         x = synth.activation_f16(self.M, self.K, seed=4)
         wq, s = synth.int8_weight_groups(self.N, self.K, seed=4)
-        t0 = time.perf_counter()
-        O.gemm_w8a16_group(x, wq, s)
-        dt = time.perf_counter() - t0
-        return self.units_per_step, dt, f"full problem M={self.M} N={self.N} K={self.K}"
+
+        def run(rows):                       # rows of W (output channels)
+            t0 = time.perf_counter()
+            O.gemm_w8a16_group(x, wq[:rows], s[:rows])
+            return time.perf_counter() - t0
+        rows = _scale_rows(run, 64, self.N, budget_s)
+        dt = run(rows)
+        frac = rows / self.N
+        return self.units_per_step * frac, dt, f"{rows} of {self.N} weight rows, M={self.M}, K={self.K}"
+
+    def sub_results(self):
+        return [("gemm_w8a16_group", f"a6 W8A16 GEMM M={self.M} N={self.N} K={self.K}", "hbm", self.dom_bytes)]
 
 
 WORKLOADS = {"w8a8_channel": ChannelW8A8, "w8a8_block": BlockW8A8, "requant": Requant, "w8a16": W8A16}
@@ -463,7 +503,95 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------------- main
 
+def _measure(wl, steps: int, warmup: int, hold_ms: float, stream, barrier, clocks=None):
+    """W warm-up steps, K timed steps back to back, then K steps with an event pair around every
+    launch.  Returns (total_ms of the back-to-back region, per-kernel mean launch ms)."""
+    import torch
+    from activation_quantized_gemm_b200 import i8q
+    nk = len(wl.kernels)
+    for i in range(warmup):
+        for k in range(nk):
+            wl.launch(i, k, stream)
+    i8q.i8q_status_check()
+    barrier()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(steps)]
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.3)
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    # Hold the stream with a device-side sleep (outside the timed region) while the host enqueues
+    # all K steps, so that host launch overhead never leaves the GPU idle inside the timed region.
+    # The timed region holds nothing but the steps' kernels: a GEMM may then overlap its start-up
+    # with the tail of the kernel before it (programmatic dependent launch).
+    torch.cuda._sleep(int(hold_ms * 1.9e6))
+    t_start.record(stream)
+    for i in range(steps):
+        for k in range(nk):
+            wl.launch(i, k, stream)
+    t_end.record(stream)
+    barrier()
+    # Per-kernel durations: the same K steps again with an event pair around every launch (the
+    # events keep each kernel from overlapping its neighbours, so these are whole launch durations).
+    torch.cuda._sleep(int(hold_ms * 1.9e6))
+    for i in range(steps):
+        ev[i][0].record(stream)
+        for k in range(nk):
+            wl.launch(i, k, stream)
+            ev[i][k + 1].record(stream)
+    barrier()
+    if clocks is not None:
+        clocks.stop()
+    i8q.i8q_status_check()
+    total_ms = t_start.elapsed_time(t_end)
+    per_kernel_ms = [sum(ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(steps)) / steps for k in range(nk)]
+    return total_ms, per_kernel_ms
+
+
+def _figure(bound: str, units: float, ms: float, peaks) -> dict:
+    """Throughput of `units` (ops for a tensor-bound kernel, bytes otherwise) in `ms`, and its
+    fraction of the measured peak."""
+    if bound == "tensor":
+        v = units / 1e12 / (ms / 1e3)
+        peak = peaks["bf16_tflops"] * INT8_PER_BF16
+        return {"value": round(v, 2), "unit": "TOPS", "frac": round(v / peak, 4)}
+    v = units / 1e9 / (ms / 1e3)
+    return {"value": round(v, 1), "unit": "GB/s", "frac": round(v / peaks["hbm_gbs"], 4)}
+
+
+# The sub-results of the default run: (name, workload, M, proj).  Each is the configured shape of
+# one more kernel of the metric; all run on one GPU after the headline step.
+SUB_WORKLOADS = [
+    ("channel_m4096", "w8a8_channel", 4096, "up"),
+    ("channel_m16", "w8a8_channel", 16, "up"),
+    ("block_up_m16", "w8a8_block", 16, "up"),
+    ("block_down_m16", "w8a8_block", 16, "down"),
+    ("requant", "requant", 0, "up"),
+    ("w8a16_m16_n12288", "w8a16", 16, "up"),
+    ("w8a16_m16_n4096", "w8a16", 16, "down"),
+]
+
+
+def _sub_entry(wl, total_ms: float, per_kernel_ms, steps: int, peaks) -> dict:
+    """Per-kernel figures of one workload plus its back-to-back step."""
+    out = {"config": wl.config["workload"], "kernels": {}}
+    step_units = 0.0
+    for (kname, label, bound, units) in wl.sub_results():
+        ms = per_kernel_ms[wl.kernels.index(kname)]
+        fig = _figure(bound, units, ms, peaks)
+        out["kernels"][kname] = {"what": label, "us": round(ms * 1e3, 2), "bound": bound, **fig}
+        step_units += units if bound == "hbm" else 0.0
+    step_ms = total_ms / steps
+    out["step_us"] = round(step_ms * 1e3, 2)
+    if all(b == "hbm" for (_, _, b, _) in wl.sub_results()):
+        fig = _figure("hbm", step_units, step_ms, peaks)
+        out["step_GBps"], out["step_frac"] = fig["value"], fig["frac"]
+    return out
+
+
 def run_ours(args):
+    import datetime
     import torch
     import torch.distributed as dist
     from activation_quantized_gemm_b200 import build
@@ -473,8 +601,12 @@ def run_ours(args):
     args.world = world
     torch.cuda.set_device(local)
     if world > 1:
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local))
-    build.build()
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=datetime.timedelta(seconds=300))
+    if rank == 0 or world == 1:
+        build.build()
+    if world > 1:
+        dist.barrier()
     wl = WORKLOADS[args.workload](args, rank)
     stream = torch.cuda.current_stream()
     nk = len(wl.kernels)
@@ -484,45 +616,8 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    for i in range(args.warmup):
-        for k in range(nk):
-            wl.launch(i, k, stream)
-    from activation_quantized_gemm_b200 import i8q
-    i8q.i8q_status_check()
-    barrier()
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    barrier()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    # Hold the stream with a device-side sleep (outside the timed region) while the host enqueues
-    # all K steps, so that host launch overhead never leaves the GPU idle inside the timed region.
-    # The timed region holds nothing but the steps' kernels: a GEMM may then overlap its start-up
-    # with the tail of the kernel before it (programmatic dependent launch).
-    torch.cuda._sleep(int(args.hold_ms * 1.9e6))
-    t_start.record(stream)
-    for i in range(args.steps):
-        for k in range(nk):
-            wl.launch(i, k, stream)
-    t_end.record(stream)
-    barrier()
-    # Per-kernel durations: the same K steps again with an event pair around every launch (the
-    # events keep each kernel from overlapping its neighbours, so these are whole launch durations).
-    torch.cuda._sleep(int(args.hold_ms * 1.9e6))
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        for k in range(nk):
-            wl.launch(i, k, stream)
-            ev[i][k + 1].record(stream)
-    barrier()
-    clocks.stop()
-    i8q.i8q_status_check()
-    total_ms = t_start.elapsed_time(t_end)
-    per_kernel_ms = [sum(ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(args.steps)) / args.steps
-                     for k in range(nk)]
+    total_ms, per_kernel_ms = _measure(wl, args.steps, args.warmup, args.hold_ms, stream, barrier, clocks)
     total_ms = max_over_ranks(total_ms, "cuda")
 
     # end to end through the public API: pinned host input -> device, step, result -> host
@@ -540,14 +635,34 @@ def run_ours(args):
     e2e_ms = e0.elapsed_time(e1)
     e2e_ms = max_over_ranks(e2e_ms, "cuda")
 
+    peaks, src = load_peaks()
+    subs = None
+    if world == 1 and not args.no_sub:
+        subs = {args.workload: _sub_entry(wl, total_ms, per_kernel_ms, args.steps, peaks)}
+        main_cfg = (args.workload, wl.config.get("M", 0), args.proj)
+        del wl.bufs
+        torch.cuda.empty_cache()
+        for (name, wname, M, proj) in SUB_WORKLOADS:
+            if (wname, M, proj) == main_cfg:
+                continue
+            sargs = argparse.Namespace(**vars(args))
+            sargs.M, sargs.proj, sargs.workload = M, proj, wname
+            swl = WORKLOADS[wname](sargs, rank)
+            t_ms, pk_ms = _measure(swl, args.sub_steps, args.warmup, args.hold_ms, stream, barrier)
+            subs[name] = _sub_entry(swl, t_ms, pk_ms, args.sub_steps, peaks)
+            del swl
+            torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import ref_cpp
         units, secs, desc = wl.oracle_sample(args.cpu_budget)
-        cpu = {"value": units / secs, "unit": wl.unit, "cores": 1, "kind": "oracle",
-               "sample": desc + f"; {secs:.2f} s of single-threaded numpy (int64 matmul does not use BLAS threads)"}
+        cpu = {"value": units / secs, "unit": wl.unit, "cores": ref_cpp.num_threads(), "kind": "oracle",
+               "host_cores": os.cpu_count(),
+               "sample": desc + f"; {secs:.2f} s of the plain C++ oracle (g++ -O2, OpenMP over "
+                                f"{ref_cpp.num_threads()} threads)"}
 
     if rank == 0:
-        peaks, src = load_peaks()
         dom_ms = per_kernel_ms[wl.kernels.index(wl.dominant)]
         if wl.dom_bound == "tensor":
             peak = peaks["bf16_tflops"] * INT8_PER_BF16
@@ -582,6 +697,13 @@ def run_ours(args):
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }
+        if subs is not None:
+            line["sub_results"] = subs
+            line["sub_results_note"] = (
+                "each entry timed in this run after the headline (its own warm-up and "
+                f"{args.sub_steps} steps, rotating >2x L2 of inputs); us = mean per-launch event time; "
+                "frac = of the measured HBM copy peak or the INT8 dense peak (bf16 burst x 2); "
+                "step_us = back-to-back step (launches overlap through programmatic dependent launch)")
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -591,10 +713,11 @@ def run_ours(args):
 def run_reference(args):
     """The CPU oracle as the reference arm: K timed steps, each a bounded sample of the workload."""
     rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    world = int(os.environ.get("WORLD_SIZE", str(max(1, args.gpus))))
     if rank != 0:
         return
     args.world = world
+    from oracle import ref_cpp
 
     cls = WORKLOADS[args.workload]
     wl = cls.__new__(cls)
@@ -618,22 +741,39 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot_s / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64/fp64",
             "data": "synthetic", "config": cfg,
-            "cpu_baseline": {"value": round(v, 6), "unit": wl.unit, "cores": 1, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": round(v, 6), "unit": wl.unit, "cores": ref_cpp.num_threads(),
+                             "host_cores": os.cpu_count(), "kind": "oracle",
+                             "sample": desc + " per step; the plain C++ oracle (OpenMP)"},
             "e2e": {"value": round(v, 6), "unit": wl.unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def _spawned_rank(rank: int, args, world: int, port: int):
+    os.environ.update({"RANK": str(rank), "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    run_ours(args)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="w8a8_channel")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="w8a8_block")
     ap.add_argument("--M", type=int, default=0, help="token rows (default: the workload's headline M)")
     ap.add_argument("--proj", choices=["up", "down"], default="up")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub", action="store_true", help="skip the per-kernel sub-results")
+    ap.add_argument("--sub-steps", type=int, default=20)
     ap.add_argument("--hold-ms", type=float, default=50.0,
                     help="device-side sleep enqueued before each timed region so the host runs ahead")
     ap.add_argument("--traffic", type=float, default=None,
@@ -643,6 +783,10 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU, spawned here (torchrun sets WORLD_SIZE itself and skips this)
+        import torch.multiprocessing as mp
+        mp.spawn(_spawned_rank, args=(args, args.gpus, _free_port()), nprocs=args.gpus, join=True)
     else:
         run_ours(args)
 

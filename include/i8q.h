@@ -75,7 +75,8 @@ i8q_status i8q_quant_act_token_group(const uint16_t* x_bf16, int64_t M, int64_t 
  * quantizer (one scale per output channel = per row of W [N][K]).
  * [R1-INT8] section 2.3, channel-wise paragraph.
  *   x_bf16 : [M][ldx] bf16, K valid columns; ldx >= K, ldx % 8 == 0.
- *   M, K   : M >= 0; K >= 0, K % 16 == 0.
+ *   M, K   : M >= 0; K >= 0, K % 8 == 0 (rows move as 16-byte vectors of 8 values; every K of
+ *            the pages' layers is a multiple of 128).
  *   xq     : [M][K] int8 output.   sx : [M] fp32 output (one scale per row).
  * M == 0 is a no-op; K == 0 writes sx = 0.
  */
@@ -125,7 +126,8 @@ i8q_status i8q_requant_fp8_to_int8_channel(const uint8_t* w_e4m3, const float* s
  *   xq  : [M][K] int8;   sx : [K/128][ld_sx] fp32 (token-contiguous, as written by
  *         i8q_quant_act_token_group); ld_sx >= M, ld_sx % 4 == 0.
  *   wq  : [N][K] int8;   sw : [ceil(N/128)][K/128] fp32.
- *   M >= 0; N >= 0, N % 8 == 0; K >= 0, K % 128 == 0.
+ *   M >= 0; N >= 0 (any N: a partial last weight block shares that block's scale and the
+ *   output columns past N are never written); K >= 0, K % 128 == 0.
  *   y   : [M][N], bf16 (out == I8Q_OUT_BF16, round to nearest even) or fp32 (I8Q_OUT_FP32).
  *   debug_partials : NULL, or [M][N][K/128] int32 receiving every P (checking aid; slower).
  * M == 0 or N == 0 is a no-op; K == 0 writes y = 0.
@@ -141,7 +143,7 @@ i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx,
  * [R1-INT8] section 2.3, channel-wise paragraph and Fig. 3 (right): a single dequantization
  * after the INT8 GEMM with the per-token and per-output-channel scales.
  *   xq : [M][K] int8;  sx : [M] fp32;  wq : [N][K] int8;  sw : [N] fp32.
- *   M >= 0; N >= 0, N % 8 == 0; K >= 0, K % 128 == 0 (127^2 * K < 2^31 keeps int32 exact).
+ *   M >= 0; N >= 0 (any N); K >= 0, K % 128 == 0 (127^2 * K < 2^31 keeps int32 exact).
  *   y_bf16 : [M][N] bf16 output (round to nearest even).
  *   debug_acc : NULL, or [M][N] int32 receiving A (checking aid).
  * M == 0 or N == 0 is a no-op; K == 0 writes y = 0.
@@ -157,7 +159,7 @@ i8q_status i8q_gemm_w8a8_channel(const int8_t* xq, const float* sx, const int8_t
  *   y[m][n] = fp16( sum_g s[n][g] * sum_{k in group g} x[m][k] * wq[n][k] )
  * with the products exact in fp32 and fp32 accumulation.
  *   x_f16 : [M][K] fp16;  wq : [N][K] int8;  s_f16 : [N][K/128] fp16 group scales.
- *   1 <= M <= 64 (decode batch); N >= 0, N % 8 == 0; K >= 0, K % 128 == 0.
+ *   1 <= M <= 64 (decode batch); N >= 0 (any N); K >= 0, K % 128 == 0.
  *   y_f16 : [M][N] fp16 output (round to nearest even).
  * M == 0 or N == 0 is a no-op; K == 0 writes y = 0; M > 64 gives I8Q_ERR_SHAPE.
  */
@@ -176,6 +178,20 @@ const char* i8q_last_error_string(void);
  * I8Q_ERR_CUDA if the stream reported an error, I8Q_OK otherwise.
  */
 i8q_status i8q_status_check(void* stream);
+
+/*
+ * Test aids for the bounded device waits (no counterpart in the pages; used by the test suite).
+ * i8q_test_set_wait_limit_ns: limit of every pipeline wait on the current device, in ns
+ *   (0 restores the default of 2 s).  Waits that drain copies already in flight keep 2 s.
+ * i8q_test_skip_accumulator_signal: armed != 0 makes the next decode-size (M <= 128) channel-wise
+ *   W8A8 GEMM launch withhold one accumulator-ready signal in one CTA, so that its epilogue's wait
+ *   expires (after the limit above), the kernel returns early, and i8q_status_check() reports
+ *   I8Q_ERR_TIMEOUT; the output of that launch is undefined.  armed == 0 disarms it.
+ * Both write a device variable synchronously (cudaMemcpyToSymbol); do not call them while
+ * kernels of this library are running.
+ */
+i8q_status i8q_test_set_wait_limit_ns(uint64_t ns);
+i8q_status i8q_test_skip_accumulator_signal(int armed);
 
 /* Library version, as major * 10000 + minor * 100 + patch. */
 int i8q_version(void);

@@ -6,6 +6,8 @@ from activation_quantized_gemm_b200 import build
 
 
 def setup_library():
+    from oracle import ref_cpp
+    ref_cpp.load()                 # the C++ oracle every GPU parity test compares with
     build.build()
     from activation_quantized_gemm_b200 import i8q
     i8q.load()

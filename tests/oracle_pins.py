@@ -316,3 +316,31 @@ def check_w8a16(gemm_w8a16_group, seed=7, M=4, N=33, K=384):
                     part += _frac(x[m, k]) * int(wq[n, k])
                 y += part * _frac(s[n, g])
             assert abs(_frac(Y[m, n]) - y) <= Fraction(1, 10 ** 14) * _frac(T[m, n]) + Fraction(1, 10 ** 300)
+
+
+def check_w8a16_bf16(gemm_w8a16_group_bf16, seed=8, M=3, N=21, K=384):
+    """bf16 activations and group scales: scale 1 reduces to a plain fp64 matmul of the bf16 values
+    (torch's bf16 decode as the library routine); random scales against exact fractions."""
+    import torch
+    rng = np.random.default_rng(seed)
+    xt = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+    xb = xt.view(torch.int16).numpy().view(np.uint16)
+    xv = xt.double().numpy()
+    wq = rng.integers(-127, 128, (N, K)).astype(np.int8)
+    one = np.full((N, K // 128), 0x3F80, np.uint16)                         # bf16 1.0
+    Y, T = gemm_w8a16_group_bf16(xb, wq, one)
+    ref = torch.from_numpy(xv) @ torch.from_numpy(wq.astype(np.float64)).T
+    assert np.allclose(Y, ref.numpy(), rtol=1e-13, atol=1e-12)
+    st = torch.from_numpy(rng.uniform(1e-4, 1e-3, (N, K // 128)).astype(np.float32)).to(torch.bfloat16)
+    sb = st.view(torch.int16).numpy().view(np.uint16)
+    sv = st.double().numpy()
+    Y, T = gemm_w8a16_group_bf16(xb, wq, sb)
+    for m in range(M):
+        for n in range(0, N, 4):
+            y = Fraction(0)
+            for g in range(K // 128):
+                part = Fraction(0)
+                for k in range(g * 128, g * 128 + 128):
+                    part += _frac(xv[m, k]) * int(wq[n, k])
+                y += part * _frac(sv[n, g])
+            assert abs(_frac(Y[m, n]) - y) <= Fraction(1, 10 ** 14) * _frac(T[m, n]) + Fraction(1, 10 ** 300)

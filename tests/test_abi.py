@@ -43,8 +43,8 @@ def test_shape_checks(lib):
     # K not a multiple of 128
     assert _st(lib, "i8q_quant_act_token_group", P, 4, 100, 100, P, P, 4, None) == 2
     assert _st(lib, "i8q_gemm_w8a8_channel", P, P, P, P, 4, 8, 200, P, None, None) == 2
-    # N not a multiple of 8
-    assert _st(lib, "i8q_gemm_w8a8_block", P, P, 4, P, P, 4, 12, 128, P, 0, None, None) == 2
+    # a2: K not a multiple of 8 (its rows move as 8-value vectors)
+    assert _st(lib, "i8q_quant_act_token", P, 4, 12, 16, P, P, None) == 2
     # negative sizes
     assert _st(lib, "i8q_quant_act_token", P, -1, 128, 128, P, P, None) == 2
     # ldx < K, ld_sx < M, ld_sx not a multiple of 4
@@ -71,6 +71,19 @@ def test_empty_problems_are_noops(lib):
     assert _st(lib, "i8q_gemm_w8a8_channel", None, None, None, None, 0, 8, 128, None, None, None) == 0
     assert _st(lib, "i8q_gemm_w8a8_block", None, None, 0, None, None, 4, 0, 128, None, 0, None, None) == 0
     assert _st(lib, "i8q_gemm_w8a16_group", None, None, None, 0, 8, 128, None, None) == 0
+
+
+def test_any_n_passes_the_shape_checks(lib):
+    """N need not be a multiple of 8 (masked tails): with no GPU such a call gets past every
+    argument check and fails only at the device (I8Q_ERR_CUDA), never with I8Q_ERR_SHAPE."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    for n in (1, 7, 129, 7170):
+        assert _st(lib, "i8q_gemm_w8a8_block", P, P, 4, P, P, 4, n, 128, P, 0, None, None) == 5
+        assert _st(lib, "i8q_gemm_w8a8_channel", P, P, P, P, 4, n, 128, P, None, None) == 5
+        assert _st(lib, "i8q_gemm_w8a16_group", P, P, P, 4, n, 128, P, None) == 5
+    assert _st(lib, "i8q_quant_act_token", P, 4, 24, 24, P, P, None) == 5
 
 
 def test_valid_call_without_device_fails_loudly(lib):

@@ -31,7 +31,9 @@ def test_reference_line_matches_gpu_arm_config(workload, kw):
     assert line["metric"] == bench.METRIC
     assert line["config"] == bench.describe(workload, args)["config"]
     assert line["unit"] == bench.WORKLOADS[workload].unit
-    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+    from oracle import ref_cpp
+    assert line["cpu_baseline"]["cores"] == ref_cpp.num_threads() >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
 
 
@@ -39,16 +41,43 @@ def test_describe_shapes():
     d = bench.describe("w8a8_block", _args("w8a8_block", M=16384))
     assert (d["M"], d["N"], d["K"]) == (16384, 18432, 7168) and d["R"] >= 1
     d = bench.describe("w8a8_block", _args("w8a8_block", proj="down"))
-    assert (d["M"], d["N"], d["K"]) == (4096, 7168, 18432)
+    assert (d["M"], d["N"], d["K"]) == (16384, 7168, 18432)
     d = bench.describe("w8a16", _args("w8a16"))
     assert (d["M"], d["N"], d["K"]) == (16, 12288, 4096)
     assert bench.describe("w8a8_channel", _args("w8a8_channel", world=4))["config"]["global_batch"] == 4 * 4096
 
 
 def test_measured_traffic_lookup():
-    traffic, src = bench.measured_traffic("w8a8_channel", {"M": 4096, "N": 7168, "K": 2048})
+    traffic, src = bench.measured_traffic("w8a16", {"M": 16, "N": 12288, "K": 4096})
     assert traffic and src.endswith(".md")
     assert bench.measured_traffic("w8a8_channel", {"M": 7, "N": 7168, "K": 2048}) == (None, None)
+
+
+def test_default_is_the_block_wise_prefill_layer():
+    import sys
+    argv = sys.argv
+    try:
+        sys.argv = ["bench.py"]
+        ap_args = None
+        import argparse
+        orig = argparse.ArgumentParser.parse_args
+
+        def grab(self, *a, **k):
+            nonlocal ap_args
+            ap_args = orig(self, *a, **k)
+            raise SystemExit(0)
+        argparse.ArgumentParser.parse_args = grab
+        try:
+            bench.main()
+        except SystemExit:
+            pass
+        finally:
+            argparse.ArgumentParser.parse_args = orig
+    finally:
+        sys.argv = argv
+    assert ap_args.workload == "w8a8_block" and ap_args.proj == "up"
+    d = bench.describe(ap_args.workload, ap_args)
+    assert (d["M"], d["N"], d["K"]) == (16384, 18432, 7168)
 
 
 def test_traffic_sources_exist():

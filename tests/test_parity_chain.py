@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 import torch
 
-import oracle as O
+from oracle import ref_cpp as O
 from activation_quantized_gemm_b200 import synth
 from criteria import check_fp32, check_half
 from gpu_util import dev, empty, host, setup_library
@@ -68,7 +68,7 @@ def test_channel_chain(q, M, D):
         xq_r, sx_r = O.quant_act_token(host(acts[i], np.uint16))
         wq_r, sw_r = O.quant_act_token(ws[i])
         Y, _ = O.gemm_w8a8_channel(xq_r, sx_r, wq_r, sw_r)
-        check_half(host(acts[i + 1], np.uint16), Y, np.abs(Y), "bf16", f"channel chain layer {i} M={M}")
+        check_half(host(acts[i + 1], np.uint16), Y, np.abs(Y), "bf16", f"channel chain layer {i} M={M}", strict=True)
 
 
 @pytest.mark.parametrize("M", [1, 16])

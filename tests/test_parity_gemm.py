@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-import oracle as O
+from oracle import ref_cpp as O
 from activation_quantized_gemm_b200 import synth
 from criteria import check_fp32, check_half
 from gpu_util import dev, empty, host, setup_library
@@ -23,7 +23,11 @@ SHAPES = [(1, 8, 128), (16, 256, 512), (7, 200, 384), (130, 264, 1024), (300, 52
           # decode kernel with 128-token padding (65..128 tokens, one CTA per SM)
           (100, 1032, 1536), (128, 264, 4096),
           # channel-wise pair-tile widths 224 and 256 (chosen by wave fill; smaller shapes take 192)
-          (200, 16384, 256), (130, 18944, 256)]
+          (200, 16384, 256), (130, 18944, 256),
+          # any N: masked tails (unaligned output rows, a partial last weight block), decode and
+          # prefill kernels
+          (1, 1, 128), (16, 7, 256), (40, 129, 512), (300, 7, 384), (257, 129, 256), (33, 7170, 512),
+          (260, 7170, 256)]
 
 
 @pytest.fixture(scope="module")
@@ -67,7 +71,7 @@ def test_channel(q, M, N, K, kind):
     torch.cuda.synchronize()
     assert np.array_equal(host(acc), A.astype(np.int32))
     T = np.abs(Y)
-    check_half(host(y, np.uint16), Y, T, "bf16", f"channel {M}x{N}x{K}")
+    check_half(host(y, np.uint16), Y, T, "bf16", f"channel {M}x{N}x{K}", strict=True)
     # the production variant (no debug output) writes the same bits
     y2 = empty((M, N), torch.int16, 0x7FC0)
     q.i8q_gemm_w8a8_channel(dev(xq), dev(sx), dev(wq), dev(sw), y2)
@@ -143,9 +147,35 @@ def test_extreme_accumulators(q, M, N, K):
     q.i8q_gemm_w8a8_block(dev(xqb), sxd, dev(wqb), dev(swb), y32, out=q.I8Q_OUT_FP32, debug_partials=dbg)
     torch.cuda.synchronize()
     assert np.array_equal(host(acc), A.astype(np.int32))
-    check_half(host(y, np.uint16), Y, np.abs(Y), "bf16", "extreme channel")
+    check_half(host(y, np.uint16), Y, np.abs(Y), "bf16", "extreme channel", strict=True)
     assert np.array_equal(host(dbg), Pb.astype(np.int32))
     check_fp32(host(y32), Yb, Tb, "extreme block")
+
+
+@pytest.mark.parametrize("M,N", [(16, 7), (70, 129), (300, 7), (260, 7170)])
+def test_ragged_n_stays_in_bounds(q, M, N):
+    """N not a multiple of 8: every output element is written exactly where it belongs and nothing
+    past the packed [M, N] output (all four kernels: decode / pair tiles, channel / block, bf16 and fp32)."""
+    K = 256
+    x, w = _inputs(M, N, K, seed=M + N)
+    xq, sx = O.quant_act_token(x)
+    wq, sw = O.quant_act_token(w)
+    Y, A = O.gemm_w8a8_channel(xq, sx, wq, sw)
+    big = empty((M * N + 96,), torch.int16, 0x1234)
+    q.i8q_gemm_w8a8_channel(dev(xq), dev(sx), dev(wq), dev(sw), big[: M * N].view(M, N))
+    xqb, sxb, wqb, swb = _block_operands(x, w)
+    Yb, Tb, Pb = O.gemm_w8a8_block(xqb, sxb, wqb, swb)
+    sxd = dev(np.ascontiguousarray(np.pad(sxb.T, ((0, 0), (0, (-M) % 4)))))
+    big16 = empty((M * N + 96,), torch.int16, 0x1234)
+    q.i8q_gemm_w8a8_block(dev(xqb), sxd, dev(wqb), dev(swb), big16[: M * N].view(M, N))
+    big32 = empty((M * N + 96,), torch.float32, 1234.5)
+    q.i8q_gemm_w8a8_block(dev(xqb), sxd, dev(wqb), dev(swb), big32[: M * N].view(M, N), out=q.I8Q_OUT_FP32)
+    torch.cuda.synchronize()
+    h, h16, h32 = host(big).view(np.uint16), host(big16).view(np.uint16), host(big32)
+    assert np.all(h[M * N:] == 0x1234) and np.all(h16[M * N:] == 0x1234) and np.all(h32[M * N:] == 1234.5)
+    check_half(h[: M * N].reshape(M, N), Y, np.abs(Y), "bf16", f"channel ragged {M}x{N}", strict=True)
+    check_half(h16[: M * N].reshape(M, N), Yb, Tb, "bf16", f"block ragged {M}x{N}")
+    check_fp32(h32[: M * N].reshape(M, N), Yb, Tb, f"block fp32 ragged {M}x{N}")
 
 
 def test_outputs_stay_in_bounds(q):

@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 import torch
 
-import oracle as O
+from oracle import ref_cpp as O
 from activation_quantized_gemm_b200 import synth
 from gpu_util import dev, empty, host, setup_library
 
@@ -61,7 +61,8 @@ def test_act_token_group_strided_input(q):
     assert np.array_equal(host(sx)[:, :M].T, sx_ref)
 
 
-@pytest.mark.parametrize("M,K", [(16, 2048), (1, 16), (300, 2048), (6, 7168), (7, 18432), (130, 4096), (5, 24576), (1001, 384)])
+@pytest.mark.parametrize("M,K", [(16, 2048), (1, 16), (300, 2048), (6, 7168), (7, 18432), (130, 4096), (5, 24576), (1001, 384),
+                                 (1, 8), (9, 24), (33, 40), (6, 1000)])
 def test_act_token(q, M, K):
     x = _edge_activations(M, K, seed=2 * M + K)
     xq_ref, sx_ref = O.quant_act_token(x)

@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 import torch
 
-import oracle as O
+from oracle import ref_cpp as O
 from activation_quantized_gemm_b200 import synth
 from criteria import check_half
 from gpu_util import dev, empty, host, setup_library
@@ -28,7 +28,8 @@ def test_w8a16(q, M, N, K):
     check_half(host(y, np.uint16), Y, T, "fp16", f"w8a16 {M}x{N}x{K}")
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 264, 16384), (3, 136, 18432), (4, 8, 256), (2, 4104, 1024)])
+@pytest.mark.parametrize("M,N,K", [(1, 264, 16384), (3, 136, 18432), (4, 8, 256), (2, 4104, 1024),
+                                   (1, 1, 128), (5, 7, 256), (16, 129, 512), (64, 4097, 1024)])
 def test_w8a16_small_batches_long_rows(q, M, N, K):
     """Small decode batches with long rows (K up to 18432: 144 groups split over clusters of up to
     8 CTAs), a single ragged tile and many tiles."""
