@@ -84,18 +84,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Waits until the phase with the given parity has completed.  Returns false (and raises the
 // device error word) if that does not happen within kWaitTimeoutNs; `abort_flag` (shared
 // memory, may be null) is polled so that one expired wait makes every other role give up fast.
+__device__ __noinline__ unsigned long long wait_limit_ns(unsigned site) {
+  return site == SITE_DRAIN ? (unsigned long long)kWaitTimeoutNs
+                            : *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned site,
                                           volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = globaltimer_ns();
-  const unsigned long long limit =
-      site == SITE_DRAIN ? (unsigned long long)kWaitTimeoutNs
-                         : *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (abort_flag && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit) {
+      const unsigned long long dt = globaltimer_ns() - t0;
+      // the limit (a global-memory read) is fetched only once a wait has lasted 100 us
+      if (dt > 100000ull && dt > wait_limit_ns(site)) {
         raise_error(site);
         if (abort_flag) *abort_flag = 1;
         return false;

@@ -38,6 +38,7 @@ namespace i8q {
 constexpr int GEMM_BM = 256;       // tokens per pair tile (MMA M, cta_group::2)
 constexpr int GEMM_BK = 128;       // K per slab (bytes of int8 = one 128B swizzle row)
 constexpr int GEMM_GROUP_M = 8;    // pair-tile rows per raster band
+constexpr int kMaxExperts = 1024;  // grouped (MoE) GEMMs: experts per call
 
 template <int BN>
 struct W8A8Cfg {
@@ -51,6 +52,9 @@ struct W8A8Cfg {
   static constexpr int BAR_BYTES = 256;
   static constexpr int EPI_STAGE_BYTES = EPI_WARPS * 32 * 80;   // per epilogue warp: 32 rows x 80 B
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + EPI_STAGE_BYTES + 1024;  // + alignment slack
+  // grouped (MoE) problems: per-expert row offsets and m-tile prefix sums, kMaxExperts + 1 each
+  static constexpr int GROUP_BYTES = 2 * (kMaxExperts + 1) * 4;
+  static constexpr int SMEM_BYTES_GROUPED = SMEM_BYTES + GROUP_BYTES;
   static_assert(2 * BN <= TMEM_COLS, "two accumulators must fit in TMEM");
   static_assert(BN % 32 == 0 && BN <= 256, "MMA N (each CTA's BN / 2 weight rows: whole 8-row groups)");
 };
@@ -58,10 +62,14 @@ struct W8A8Cfg {
 struct W8A8Args {
   const float* sx;      // channel: [M]; block: [KB][ld_sx]
   int64_t ld_sx;
-  const float* sw;      // channel: [N]; block: [ceil(N/128)][KB]
+  const float* sw;      // channel: [N]; block: [ceil(N/128)][KB]  (grouped: one such array per expert)
   int M, N, K;
   void* y;              // [M][N] bf16 or fp32
   int32_t* dbg;         // channel: [M][N] accumulators; block: [M][N][KB] slab partials
+  const int32_t* off;   // grouped only: [E + 1] row offsets, expert e owns rows off[e] .. off[e+1]-1
+  int E;                // grouped only: number of experts (weights [E][N][K])
+  int8_t* qx_out;       // fused quantization only (nullable): [M][K] int8 codes of the activations
+  float* qs_out;        // fused quantization only (nullable): [K/128][ld_sx] group scales
 };
 
 // ------------------------------------------------------------------ pair-wide PTX wrappers ----
@@ -156,6 +164,73 @@ __device__ __forceinline__ void gemm_tile_coords(int t, int Mt, int Nt, int& mb,
   nb = idx / rows;
 }
 
+// Grouped (MoE) tables, built by one warp after the dependency wait (the offsets may have been
+// written by the kernel before): s_off[e] = the offsets made non-decreasing and clamped to [0, M]
+// (so that no row outside [0, M) is ever touched, whatever the caller passed), s_pre[e] = the
+// number of 256-row m-tiles of experts 0 .. e-1.  Global m-tile g belongs to the largest e with
+// s_pre[e] <= g (experts without tokens own no m-tile).
+__device__ __forceinline__ void build_group_tables(const int32_t* __restrict__ off, int E, int M, int* s_off,
+                                                   int* s_pre, int lane) {
+  const int n = E + 1;
+  const int chunk = (n + 31) / 32;
+  const int b = min(n, lane * chunk), e_ = min(n, b + chunk);
+  int mx = 0;
+  for (int i = b; i < e_; ++i) {
+    const int v = min(max(__ldg(off + i), 0), M);
+    s_off[i] = v;
+    mx = max(mx, v);
+  }
+  // exclusive prefix max over the lanes' chunks, then a running max inside the chunk
+  int incl = mx;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+    if (lane >= d) incl = max(incl, o);
+  }
+  int run = __shfl_up_sync(0xFFFFFFFFu, incl, 1);
+  if (lane == 0) run = 0;
+  for (int i = b; i < e_; ++i) {
+    run = max(run, s_off[i]);
+    s_off[i] = run;
+  }
+  __syncwarp();
+  // m-tiles per expert, exclusive prefix sum
+  int cnt = 0;
+  for (int i = b; i < e_ && i < E; ++i) cnt += (s_off[i + 1] - s_off[i] + GEMM_BM - 1) / GEMM_BM;
+  int inc = cnt;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xFFFFFFFFu, inc, d);
+    if (lane >= d) inc += o;
+  }
+  int pre = inc - cnt;
+  for (int i = b; i < e_; ++i) {
+    s_pre[i] = pre;
+    if (i < E) pre += (s_off[i + 1] - s_off[i] + GEMM_BM - 1) / GEMM_BM;
+  }
+  __syncwarp();
+}
+
+// Rows of global m-tile g: expert e, first row, one past the last row of the expert.
+template <bool GROUPED>
+__device__ __forceinline__ void tile_rows(int g, int M, const int* s_off, const int* s_pre, int E, int& e,
+                                          int& row0, int& row_end) {
+  if constexpr (!GROUPED) {
+    e = 0;
+    row0 = g * GEMM_BM;
+    row_end = M;
+  } else {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_pre[mid] <= g) lo = mid; else hi = mid;
+    }
+    e = lo;
+    row0 = s_off[lo] + (g - s_pre[lo]) * GEMM_BM;
+    row_end = s_off[lo + 1];
+  }
+}
+
 // fp32 bits 0x4B400000 = 1.5 * 2^23 = 12582912.  An int32 accumulator that starts from these bits
 // holds 0x4B400000 + P after the MMA adds P; for |P| < 2^22 those are exactly the bits of the
 // float 12582912 + P, so subtracting 12582912 recovers P exactly.
@@ -185,16 +260,17 @@ __device__ __forceinline__ void store_row8(void* y, bool f32out, int64_t off, co
 // columns nc .. nc + W - 1 (W = 16 or 32) of row m_base + l as bf16 pairs.  The 32 rows go through
 // a 32 x 80-byte staging slab in shared memory (80-byte rows: conflict-free for row-wise writes and
 // column-wise reads), then each store instruction writes 8 rows x 64 contiguous bytes instead of
-// 16 bytes of 32 different rows (half-filled sectors).  When N % 8 != 0 the rows of y are not
-// 16-byte aligned: every element is then stored on its own (lane = column), masked at N.
+// 16 bytes of 32 different rows (half-filled sectors).  When N % 8 != 0 (ALIGNED false) the rows of
+// y are not 16-byte aligned: every element is then stored on its own (lane = column), masked at N.
+template <bool ALIGNED>
 __device__ __forceinline__ void store_rows_bf16(uint8_t* stg, int lane, const uint32_t (&p)[16], int W, uint16_t* y,
-                                                int N, int m_base, int M, int nc, bool nvec) {
+                                                int N, int m_base, int M, int nc) {
   uint4* srow = reinterpret_cast<uint4*>(stg + lane * 80);
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     if (q * 8 < W) srow[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
   __syncwarp();
-  if (nvec) {
+  if constexpr (ALIGNED) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int r = i * 8 + (lane & 7), c = lane >> 3;
@@ -204,7 +280,6 @@ __device__ __forceinline__ void store_rows_bf16(uint8_t* stg, int lane, const ui
     }
   } else {
     const int n = nc + lane;
-#pragma unroll 4
     for (int r = 0; r < 32; ++r) {
       const int m = m_base + r;
       if (lane < W && m < M && n < N) y[(int64_t)m * N + n] = reinterpret_cast<const uint16_t*>(stg + r * 80)[lane];
@@ -218,7 +293,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int BN, bool BLOCKWISE, bool OUT_F32, bool DEBUG>
+template <int BN, bool BLOCKWISE, bool OUT_F32, bool DEBUG, bool GROUPED = false, bool ALIGNED = true>
 __global__ void __launch_bounds__(384, 1)
     k_gemm_w8a8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const W8A8Args args) {
@@ -243,9 +318,17 @@ __global__ void __launch_bounds__(384, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int M = args.M, N = args.N, K = args.K;
-  const int Mt = (M + GEMM_BM - 1) / GEMM_BM, Nt = (N + BN - 1) / BN, KB = K / GEMM_BK;
-  const int num_tiles = Mt * Nt;
-  const bool nvec = (N & 7) == 0;   // rows of y, sw and the debug outputs allow vector accesses
+  const int Nt = (N + BN - 1) / BN, KB = K / GEMM_BK;
+  int Mt = (M + GEMM_BM - 1) / GEMM_BM;   // grouped: set from the expert offsets below
+  int num_tiles = Mt * Nt;
+  // ALIGNED (N % 8 == 0, chosen by the host): rows of y, sw and the debug outputs allow vector
+  // accesses.  A compile-time choice: a run-time test in the epilogue cost 10% at K = 2048.
+  constexpr bool nvec = ALIGNED;
+  int* s_off = reinterpret_cast<int*>(sStage + C::EPI_STAGE_BYTES);   // grouped tables
+  int* s_pre = s_off + (kMaxExperts + 1);
+  const int E = GROUPED ? args.E : 1;
+  // per-expert stride of the weight scales: channel [E][N], block [E][ceil(N/128)][KB]
+  const int64_t sw_estride = BLOCKWISE ? (int64_t)((N + 127) / 128) * KB : (int64_t)N;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -263,7 +346,7 @@ __global__ void __launch_bounds__(384, 1)
   // The kernel may be launched while the preceding kernel (typically the activation quantizer) is
   // still running: until grid_dependency_wait() it touches no global memory except L2 prefetches of
   // the weight slabs of its first tile.
-  if (warp == 0 && lane == 0 && pair < num_tiles) {
+  if (!GROUPED && warp == 0 && lane == 0 && pair < num_tiles) {
     int mb, nb;
     gemm_tile_coords(pair, Mt, Nt, mb, nb);
     for (int kb = 0; kb < KB && kb < C::STAGES; ++kb)
@@ -278,6 +361,12 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   grid_dependency_wait();
+  if constexpr (GROUPED) {
+    if (warp == 2) build_group_tables(args.off, E, M, s_off, s_pre, lane);
+    __syncthreads();
+    Mt = s_pre[E];
+    num_tiles = Mt * Nt;
+  }
 
   if (warp < 4) {
     setmaxnreg_dec<24>();
@@ -288,10 +377,11 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t expected = 0, exp_parity = 0;   // leader: stages whose completion it expects
       bool ok = true;
       for (int t = pair; ok && t < num_tiles; t += npairs) {
-        int mb, nb;
+        int mb, nb, e, row0, row_end;
         gemm_tile_coords(t, Mt, Nt, mb, nb);
-        const int arow = mb * GEMM_BM + (int)rank * 128;
-        const int brow = nb * BN + (int)rank * HALF;
+        tile_rows<GROUPED>(mb, M, s_off, s_pre, E, e, row0, row_end);
+        const int arow = row0 + (int)rank * 128;
+        const int brow = e * N + nb * BN + (int)rank * HALF;   // grouped: W is [E * N][K]
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, SITE_EMPTY, abort_flag)) { ok = false; break; }
           if (leader) {
@@ -383,11 +473,13 @@ __global__ void __launch_bounds__(384, 1)
     }
 
     for (int t = pair; t < num_tiles; t += npairs) {
-      int mb, nb;
+      int mb, nb, e, row0, row_end;
       gemm_tile_coords(t, Mt, Nt, mb, nb);
-      const int m = mb * GEMM_BM + row;
+      tile_rows<GROUPED>(mb, M, s_off, s_pre, E, e, row0, row_end);
+      const int m = row0 + row;
       const int n0 = nb * BN + h * HALF;           // first column of this warp's half
-      const bool row_ok = m < M;
+      const bool row_ok = m < row_end;
+      const float* swp = args.sw + (GROUPED ? (int64_t)e * sw_estride : 0);
       if constexpr (!BLOCKWISE) {
         const uint32_t acc = acc_iter & 1;
         if (!warp_wait(&tfull[acc], (acc_iter >> 1) & 1, SITE_TMEM_FULL, abort_flag)) break;
@@ -401,17 +493,17 @@ __global__ void __launch_bounds__(384, 1)
             const int n = nc + g * 8;
             if (g * 8 < W) {
               float ws[8];
-              if (nvec) {
+              if constexpr (nvec) {
                 float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
                 if (n < N) {
-                  w0 = __ldg(reinterpret_cast<const float4*>(args.sw + n));
-                  w1 = __ldg(reinterpret_cast<const float4*>(args.sw + n + 4));
+                  w0 = __ldg(reinterpret_cast<const float4*>(swp + n));
+                  w1 = __ldg(reinterpret_cast<const float4*>(swp + n + 4));
                 }
                 ws[0] = w0.x; ws[1] = w0.y; ws[2] = w0.z; ws[3] = w0.w;
                 ws[4] = w1.x; ws[5] = w1.y; ws[6] = w1.z; ws[7] = w1.w;
               } else {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) ws[j] = n + j < N ? __ldg(args.sw + n + j) : 0.f;
+                for (int j = 0; j < 8; ++j) ws[j] = n + j < N ? __ldg(swp + n + j) : 0.f;
               }
               float v[8];
 #pragma unroll
@@ -420,7 +512,7 @@ __global__ void __launch_bounds__(384, 1)
               for (int j = 0; j < 4; ++j) pk[g * 4 + j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
               if constexpr (DEBUG) {
                 if (row_ok && n < N) {
-                  if (nvec) {
+                  if constexpr (nvec) {
                     int4* dp = reinterpret_cast<int4*>(args.dbg + (int64_t)m * N + n);
                     dp[0] = make_int4(r[g * 8 + 0], r[g * 8 + 1], r[g * 8 + 2], r[g * 8 + 3]);
                     dp[1] = make_int4(r[g * 8 + 4], r[g * 8 + 5], r[g * 8 + 6], r[g * 8 + 7]);
@@ -433,7 +525,7 @@ __global__ void __launch_bounds__(384, 1)
               }
             }
           }
-          store_rows_bf16(stg, lane, pk, W, reinterpret_cast<uint16_t*>(args.y), N, m - lane, M, nc, nvec);
+          store_rows_bf16<nvec>(stg, lane, pk, W, reinterpret_cast<uint16_t*>(args.y), N, m - lane, row_end, nc);
         };
 #pragma unroll 1
         for (int c = 0; c < HALF / 32; ++c) {
@@ -459,7 +551,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int j = 0; j < HALF / 2; ++j) sum[j] = make_float2(0.f, 0.f);
         bool ok = true;
         const bool live = row_ok && n0 < N;              // this row and weight block exist
-        const float* swrow = args.sw + (int64_t)(n0 / 128) * KB;
+        const float* swrow = swp + (int64_t)(n0 / 128) * KB;
         // raw scales of the next slab are loaded one slab ahead; the product is formed when used
         float sx_next = 0.f, sw_next = 0.f;
         if (KB > 0 && live) {
@@ -518,7 +610,7 @@ __global__ void __launch_bounds__(384, 1)
                   v[2 * j] = sum[g * 4 + j].x;
                   v[2 * j + 1] = sum[g * 4 + j].y;
                 }
-                if (nvec) {
+                if constexpr (nvec) {
                   store_row8(args.y, true, (int64_t)m * N + n, v);
                 } else {
 #pragma unroll
@@ -534,7 +626,8 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(sum[c * 16 + j].x, sum[c * 16 + j].y);
-            store_rows_bf16(stg, lane, pk, 32, reinterpret_cast<uint16_t*>(args.y), N, m - lane, M, n0 + c * 32, nvec);
+            store_rows_bf16<nvec>(stg, lane, pk, 32, reinterpret_cast<uint16_t*>(args.y), N, m - lane, row_end,
+                                  n0 + c * 32);
           }
         }
       }

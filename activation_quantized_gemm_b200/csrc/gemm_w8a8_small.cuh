@@ -16,12 +16,22 @@
 //   last warp   TMEM allocation and MMA issue (4 x tcgen05.mma per slab).
 // Two CTAs share an SM for up to 64 tokens (rings of 4..6 stages each), one CTA for 128 (TMEM and
 // registers); the launch keeps all CTAs in one wave.
+//
+// FUSEDQ (block-wise, up to 64 tokens): the activations arrive as bf16 and are quantized inside
+// the GEMM, per token and 128-wide K group, as "DeepSeek R1 INT8 quantization practice on SGLang"
+// section 2.3 prescribes ("quantized online per token-group").  The TMA warp stages the bf16 slab
+// [MP x 128] next to the weight slab; quantizer warps turn it into the int8 operand (128B-swizzled,
+// as TMA would have written it) and the group scales, with the same device code as the stand-alone
+// per-token-group quantizer, so codes and scales are bit-identical to it.  Every CTA quantizes the
+// slabs of its own K range (tiles over N repeat that small amount of work instead of a separate
+// launch and an HBM round trip of the int8 activations).
 #pragma once
 
 #include <cuda_bf16.h>
 
 #include "common.cuh"
 #include "gemm_w8a16.cuh"   // cluster helpers
+#include "quant.cuh"        // the quantizer (fused variant)
 
 namespace i8q {
 
@@ -29,11 +39,17 @@ constexpr int W8A8_SMALL_MAX_M = 128;
 
 // CPS CTAs share an SM; the stage ring fills the rest of its shared memory: under full streaming
 // load a weight slab takes about 2 us to arrive, so an SM needs of the order of 100 KB in flight.
-template <int MP, bool BLOCKWISE, int CPS>
+template <int MP, bool BLOCKWISE, int CPS, bool FUSEDQ = false>
 struct W8A8SmallCfg {
   static constexpr int W_BYTES = 128 * 128;
   static constexpr int X_BYTES = MP * 128;
   static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+  // fused: the bf16 activation slab has its own ring, freed as soon as the quantizers have read it
+  static constexpr int XB_HALF = MP * 128;                // one 64-column half of the bf16 slab
+  static constexpr int XB_BYTES = 2 * XB_HALF;
+  static constexpr int XR = FUSEDQ ? 2 : 0;               // bf16 ring stages
+  static constexpr int XRING_BYTES = XR * XB_BYTES;
+  static constexpr int QW = FUSEDQ ? (MP <= 32 ? 1 : 2) : 0;   // quantizer warps
   static constexpr int NBUF = BLOCKWISE ? 4 : 1;          // slab accumulators in TMEM
   static constexpr int TMEM_NEED = NBUF * MP;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
@@ -42,10 +58,12 @@ struct W8A8SmallCfg {
   // quarter) so that the per-slab fold of 128 columns is split over twice the threads
   static constexpr int EW = MP >= 128 ? 8 : 4;
   static constexpr int MPW = MP / (EW / 4);              // token columns per epilogue thread
-  static constexpr int NUM_THREADS = 32 * (EW + 2);      // + TMA warp + MMA warp
-  static constexpr int BAR_BYTES = 512;
+  static constexpr int NUM_THREADS = 32 * (EW + 2 + QW);   // + TMA warp + MMA warp (+ quantizers)
+  static constexpr int BAR_BYTES = FUSEDQ ? 1024 : 512;
   static constexpr int RING_BYTES = EW * 2 * MPW * 4;    // block-wise scale-product rings, one per epilogue warp
-  static constexpr int FIXED_BYTES = BAR_BYTES + RING_BYTES + 1024;   // + 1024-byte alignment slack
+  static constexpr int QR = 16 + NBUF;                   // fused: ring of per-token scales, >= STAGES + NBUF
+  static constexpr int QSX_BYTES = FUSEDQ ? QR * MP * 4 : 0;
+  static constexpr int FIXED_BYTES = XRING_BYTES + BAR_BYTES + RING_BYTES + QSX_BYTES + 1024;   // + alignment slack
   static constexpr int SM_SMEM = 233472, CTA_RESERVED = 1024, CTA_MAX = 232448;
   static constexpr int BUDGET = (SM_SMEM / CPS - CTA_RESERVED) < CTA_MAX ? (SM_SMEM / CPS - CTA_RESERVED) : CTA_MAX;
   static constexpr int STAGES_FIT = (BUDGET - FIXED_BYTES) / STAGE_BYTES;
@@ -56,7 +74,53 @@ struct W8A8SmallCfg {
   static_assert(STAGES >= 4, "stage ring");
   static_assert(MP * 128 * 4 <= STAGES * STAGE_BYTES, "reduction tile must fit in the stage buffers");
   static_assert(CPS * (SMEM_BYTES + CTA_RESERVED) <= SM_SMEM && SMEM_BYTES <= CTA_MAX, "shared memory");
+  static_assert(!FUSEDQ || (BLOCKWISE && MP <= 64), "fused quantization: block-wise, up to 64 tokens");
+  static_assert(STAGE_BYTES % 1024 == 0, "128B-swizzled buffers stay 1024-byte aligned");
+  static_assert(QR >= STAGES + NBUF, "scale ring deeper than the lead of the quantizer over the epilogue");
 };
+
+// Fused quantizer: quantize the bf16 activation slab of one stage (two 128B-swizzled halves of
+// [MP rows x 64 bf16]) into the int8 operand (128B-swizzled [MP rows x 128]) and the per-token
+// group scales.  Warp qi handles tokens [qi * MP / QW, (qi + 1) * MP / QW); LPT lanes share a token.
+template <int MP, int QW>
+__device__ __forceinline__ void quantize_slab(const uint8_t* xb, uint8_t* xq, float* qs, int qi, int lane,
+                                              int8_t* qx_out, float* qs_out, int M, int K, int kb,
+                                              int64_t ld_qs) {
+  constexpr int TPW = MP / QW;                       // tokens per quantizer warp
+  constexpr int LPT = TPW >= 32 ? 1 : 32 / TPW;      // lanes per token
+  constexpr int PASSES = TPW >= 32 ? TPW / 32 : 1;
+  constexpr int CPL = 16 / LPT;                      // 8-value bf16 chunks per lane (of 16 per row)
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps) {
+    const int m = qi * TPW + ps * 32 + lane / LPT;
+    const int part = lane % LPT;
+    uint4 v[CPL];
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) {
+      const int c = part * CPL + i;                  // chunk of the row: K offset 8c
+      const int h = c >> 3, cc = c & 7;
+      v[i] = *reinterpret_cast<const uint4*>(xb + h * (MP * 128) + m * 128 + ((cc ^ (m & 7)) << 4));
+    }
+    uint32_t ab = 0;
+#pragma unroll
+    for (int i = 0; i < CPL; ++i) ab = max_u16x2(ab, absmax_bits_x8(v[i]));
+#pragma unroll
+    for (int d = 1; d < LPT; d <<= 1) ab = max_u16x2(ab, __shfl_xor_sync(FULL_MASK, ab, d));
+    const QScale q = make_qscale(bits_to_absmax(ab));
+#pragma unroll
+    for (int i = 0; i < CPL; i += 2) {
+      const uint2 lo = quant_bf16x8(v[i], q, true), hi = quant_bf16x8(v[i + 1], q, true);
+      const int c16 = (part * CPL + i) >> 1;         // 16-byte int8 chunk of the row
+      *reinterpret_cast<uint4*>(xq + m * 128 + ((c16 ^ (m & 7)) << 4)) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+      if (qx_out != nullptr && m < M)
+        *reinterpret_cast<uint4*>(qx_out + (int64_t)m * K + kb * 128 + c16 * 16) = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    }
+    if (part == 0) {
+      qs[m] = q.s;
+      if (qs_out != nullptr && m < M) qs_out[(int64_t)kb * ld_qs + m] = q.s;
+    }
+  }
+}
 
 __device__ __forceinline__ int4 ld_dsmem_s32x4(uint32_t local_addr, uint32_t rank) {
   uint32_t remote;
@@ -75,22 +139,27 @@ __device__ __forceinline__ void tmem_ld_ch(uint32_t taddr, uint32_t (&r)[CH]) {
     tmem_ld32(taddr, r);
 }
 
-template <int MP, bool BLOCKWISE, int CPS, bool OUT_F32, bool DEBUG>
-__global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS, CPS)
+template <int MP, bool BLOCKWISE, int CPS, bool OUT_F32, bool DEBUG, bool FUSEDQ = false>
+__global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS, FUSEDQ>::NUM_THREADS, CPS)
     k_gemm_w8a8_small(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                       const W8A8Args args) {
-  using C = W8A8SmallCfg<MP, BLOCKWISE, CPS>;
+  using C = W8A8SmallCfg<MP, BLOCKWISE, CPS, FUSEDQ>;
   constexpr int EW = C::EW, MPW = C::MPW;
   constexpr int CH = MPW < 32 ? MPW : 32;   // TMEM columns per load
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* xring = smem + C::STAGES * C::STAGE_BYTES;     // fused: bf16 activation slabs
+  uint64_t* full = reinterpret_cast<uint64_t*>(xring + C::XRING_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + C::NBUF;
   uint64_t* done = tempty + C::NBUF;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* xfull = done + 1;                 // fused: bf16 activation slab landed (ring of XR)
+  uint64_t* xempty = xfull + C::XR;           // fused: bf16 slab read by the quantizers
+  uint64_t* qready = xempty + C::XR;          // fused: int8 operand and scales of the stage written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(FUSEDQ ? qready + C::STAGES : done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* qsx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES + C::RING_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = args.M, N = args.N, K = args.K;
@@ -115,6 +184,13 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS,
       mbar_init(&tempty[b], EW);
     }
     mbar_init(done, 1);
+    if constexpr (FUSEDQ) {
+      for (int r = 0; r < C::XR; ++r) {
+        mbar_init(&xfull[r], 1);
+        mbar_init(&xempty[r], C::QW);
+      }
+      for (int st = 0; st < C::STAGES; ++st) mbar_init(&qready[st], C::QW);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     for (int j = 0; j < nslab && j < C::STAGES; ++j) tma_prefetch_l2_2d(&tmW, (kb0 + j) * 128, n0);
@@ -139,6 +215,28 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS,
   }
 
   if (warp == EW) {
+    if constexpr (FUSEDQ) {
+     if (lane == 1) {
+      // bf16 activation ring (fused): waits only for the quantizers
+      uint32_t filled = 0, par = 0;
+      bool ok = true;
+      for (int j = 0; j < nslab; ++j) {
+        const int r = j % C::XR;
+        const uint32_t ph = (j / C::XR) & 1;
+        if (!mbar_wait(&xempty[r], ph ^ 1, SITE_EMPTY, abort_flag)) { ok = false; break; }
+        uint8_t* xb = xring + r * C::XB_BYTES;
+        const int kk = (kb0 + j) * 128;
+        mbar_arrive_expect_tx(&xfull[r], C::XB_BYTES);
+        tma_load_2d(xb, &tmX, &xfull[r], kk, 0);
+        tma_load_2d(xb + C::XB_HALF, &tmX, &xfull[r], kk + 64, 0);
+        filled |= 1u << r;
+        par = (par & ~(1u << r)) | (ph << r);
+      }
+      if (!ok)
+        for (int r = 0; r < C::XR; ++r)
+          if (filled & (1u << r)) mbar_wait(&xfull[r], (par >> r) & 1u, SITE_DRAIN, nullptr);
+     }
+    }
     if (lane == 0) {
       uint32_t filled = 0, par = 0;
       bool ok = true;
@@ -148,9 +246,14 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS,
         if (!mbar_wait(&empty[s], ph ^ 1, SITE_EMPTY, abort_flag)) { ok = false; break; }
         uint8_t* st = smem + s * C::STAGE_BYTES;
         const int kk = (kb0 + j) * 128;
-        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-        tma_load_2d(st, &tmW, &full[s], kk, n0);
-        tma_load_2d(st + C::W_BYTES, &tmX, &full[s], kk, 0);
+        if constexpr (FUSEDQ) {          // the int8 activations are written by the quantizers
+          mbar_arrive_expect_tx(&full[s], C::W_BYTES);
+          tma_load_2d(st, &tmW, &full[s], kk, n0);
+        } else {
+          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+          tma_load_2d(st, &tmW, &full[s], kk, n0);
+          tma_load_2d(st + C::W_BYTES, &tmX, &full[s], kk, 0);
+        }
         filled |= 1u << s;
         par = (par & ~(1u << s)) | (ph << s);
       }
@@ -169,6 +272,7 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS,
           if (!mbar_wait(&tempty[b], ((j / C::NBUF) & 1) ^ 1, SITE_TMEM_EMPTY, abort_flag)) break;
         }
         if (!mbar_wait(&full[s], ph, SITE_FULL, abort_flag)) break;
+        if (FUSEDQ && !mbar_wait(&qready[s], ph, SITE_CONVERT, abort_flag)) break;
         tc_fence_after();
         const uint32_t w0 = smem_u32(smem + s * C::STAGE_BYTES);
         const uint32_t x0 = w0 + C::W_BYTES;
@@ -188,6 +292,27 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS,
       }
       tc_commit(done);
       mbar_wait(done, 0, SITE_DRAIN, nullptr);
+    }
+  } else if (FUSEDQ && warp >= EW + 2) {
+    // quantizers: bf16 activation slab -> int8 operand + per-token group scales (see quantize_slab)
+    if constexpr (FUSEDQ) {
+      const int qi = warp - (EW + 2);
+      for (int j = 0; j < nslab; ++j) {
+        const int s = j % C::STAGES, r = j % C::XR;
+        if (!warp_wait(&xfull[r], (j / C::XR) & 1, SITE_FULL, abort_flag)) break;
+        // the int8 operand buffer of stage s is free once the MMAs of slab j - STAGES are done
+        if (!warp_wait(&empty[s], ((j / C::STAGES) & 1) ^ 1, SITE_EMPTY, abort_flag)) break;
+        quantize_slab<MP, C::QW>(xring + r * C::XB_BYTES, smem + s * C::STAGE_BYTES + C::W_BYTES,
+                                 qsx + (j % C::QR) * MP, qi, lane, blockIdx.x == 0 ? args.qx_out : nullptr,
+                                 blockIdx.x == 0 ? args.qs_out : nullptr, M, K, kb0 + j, args.ld_sx);
+        // generic-proxy reads and writes of shared memory before the tensor core and TMA touch it
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&xempty[r]);
+          mbar_arrive(&qready[s]);
+        }
+      }
     }
   } else {
     // epilogue: thread = weight row n0 + 32 * (warp % 4) + lane (TMEM lane quarter = warp % 4),
@@ -213,15 +338,17 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS,
       // shared memory: lane l loads token l (and l + 32) of slab j + 1 while slab j is folded, so
       // the global-load latency is hidden behind one slab of streaming.
       const float* swrow = args.sw + (int64_t)(n0 / 128) * KB;
-      float* ring = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES) + warp * 2 * MPW;
+      float* ring = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES) + warp * 2 * MPW;
       constexpr int PER_LANE = (MPW + 31) / 32;
       float nsx[PER_LANE], nsw = 0.f;
       auto load_scales = [&](int kb) {
         nsw = __ldg(swrow + kb);
+        if constexpr (!FUSEDQ) {
 #pragma unroll
-        for (int i = 0; i < PER_LANE; ++i) {
-          const int m = cb + lane + 32 * i;
-          nsx[i] = (lane + 32 * i < MPW && m < M) ? __ldg(args.sx + (int64_t)kb * args.ld_sx + m) : 0.f;
+          for (int i = 0; i < PER_LANE; ++i) {
+            const int m = cb + lane + 32 * i;
+            nsx[i] = (lane + 32 * i < MPW && m < M) ? __ldg(args.sx + (int64_t)kb * args.ld_sx + m) : 0.f;
+          }
         }
       };
       if (nslab > 0) load_scales(kb0);
@@ -229,6 +356,15 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS>::NUM_THREADS,
         const int b = j % C::NBUF;
         const int kb = kb0 + j;
         float* slot = ring + (j & 1) * MPW;
+        if constexpr (FUSEDQ) {
+          // token scales of slab j come from the quantizer warps through shared memory
+          if (!warp_wait(&qready[j % C::STAGES], (j / C::STAGES) & 1, SITE_CONVERT, abort_flag)) break;
+#pragma unroll
+          for (int i = 0; i < PER_LANE; ++i) {
+            const int m = cb + lane + 32 * i;
+            nsx[i] = (lane + 32 * i < MPW && m < M) ? qsx[(j % C::QR) * MP + m] : 0.f;
+          }
+        }
 #pragma unroll
         for (int i = 0; i < PER_LANE; ++i)
           if (lane + 32 * i < MPW) slot[lane + 32 * i] = nsx[i] * nsw;

@@ -180,6 +180,7 @@ static i8q_status ensure_smem(Kern k, int bytes) {
 }
 
 static constexpr int64_t kMaxDim = (int64_t)1 << 30;
+static constexpr int64_t kFusedQuantMaxM = 64;   // decode batches (see i8q_gemm_w8a8_block_fused_quant)
 
 // Resident CTAs per SM of a kernel at a block size (queried once per kernel and block size).
 template <typename Kern>
@@ -295,10 +296,10 @@ static i8q_status gemm_w8a8_common_checks(const int8_t* xq, const float* sx, con
   return I8Q_OK;
 }
 
-template <int BN, bool BLOCKWISE, bool F32, bool DBG>
+template <int BN, bool BLOCKWISE, bool F32, bool DBG, bool ALIGNED = true>
 static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms, cudaStream_t s) {
   using C = W8A8Cfg<BN>;
-  auto kern = k_gemm_w8a8<BN, BLOCKWISE, F32, DBG>;
+  auto kern = k_gemm_w8a8<BN, BLOCKWISE, F32, DBG, false, ALIGNED>;
   const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
   if (attr) return attr;
   CUtensorMap ta, tb;
@@ -325,6 +326,55 @@ static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args
   cfg.attrs = at;
   cfg.numAttrs = 2;
   I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, a));
+  return I8Q_OK;
+}
+
+// Grouped (MoE) problems: the pair-tile kernel with the expert map.  The number of m-tiles is
+// known only on the device (the offsets are device data), so the grid covers the worst case:
+// every expert may add one partial m-tile, ceil(M / 256) + E m-tiles in all.
+template <bool BLOCKWISE, bool F32, bool DBG>
+static i8q_status launch_w8a8_grouped(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms,
+                                      cudaStream_t s) {
+  constexpr int BN = 256;
+  using C = W8A8Cfg<BN>;
+  auto kern = a.N % 8 == 0 ? k_gemm_w8a8<BN, BLOCKWISE, F32, DBG, true, true>
+                           : k_gemm_w8a8<BN, BLOCKWISE, F32, DBG, true, false>;
+  const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES_GROUPED);
+  if (attr) return attr;
+  CUtensorMap ta, tb;
+  i8q_status st = make_tmap_2d(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, a.K, 128, GEMM_BK,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  st = make_tmap_2d(&tb, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * a.N, a.K, a.K, BN / 2, GEMM_BK,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  const int64_t tiles = (cdiv(a.M, GEMM_BM) + a.E) * cdiv(a.N, BN);
+  const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES_GROUPED;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see grid_dependency_wait()
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, a));
+  return I8Q_OK;
+}
+
+static i8q_status grouped_checks(const int32_t* off, int64_t E, int64_t M, int64_t N, int64_t K) {
+  I8Q_REQUIRE(E >= 1 && E <= kMaxExperts, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(E * N < ((int64_t)1 << 31), I8Q_ERR_SHAPE);   // row coordinates of the stacked weights
+  (void)M;
+  (void)K;
+  I8Q_REQUIRE(off, I8Q_ERR_NULL);
+  I8Q_REQUIRE(aligned16(off), I8Q_ERR_ALIGN);
   return I8Q_OK;
 }
 
@@ -364,6 +414,50 @@ static i8q_status launch_w8a8_small_mp(const int8_t* xq, const int8_t* wq, const
   return I8Q_OK;
 }
 
+// Block-wise GEMM with the activation quantization fused in (decode batches, M <= 64): the decode
+// kernel with quantizer warps; X arrives as bf16 through its own TMA map.
+template <int MP, bool F32>
+static i8q_status launch_w8a8_fused_mp(const uint16_t* x, int64_t ldx, const int8_t* wq, const W8A8Args& a, int sms,
+                                       cudaStream_t s) {
+  constexpr int CPS = MP <= 32 ? 2 : 1;
+  using C = W8A8SmallCfg<MP, true, CPS, true>;
+  auto kern = k_gemm_w8a8_small<MP, true, CPS, F32, false, true>;
+  const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
+  if (attr) return attr;
+  CUtensorMap tw, tx;
+  i8q_status st = make_tmap_2d(&tw, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, a.K, 128, 128,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  st = make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.K, ldx, MP, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st) return st;
+  const int64_t tiles = cdiv(a.N, 128);
+  const int splits = w8a8_small_splits(tiles, a.K / 128, sms, CPS);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits, 1);
+  cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 1;
+  at[0].val.clusterDim.y = (unsigned)splits;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see grid_dependency_wait()
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, tw, tx, a));
+  return I8Q_OK;
+}
+
+template <bool F32>
+static i8q_status launch_w8a8_fused(const uint16_t* x, int64_t ldx, const int8_t* wq, const W8A8Args& a, int sms,
+                                    cudaStream_t s) {
+  if (a.M <= 16) return launch_w8a8_fused_mp<16, F32>(x, ldx, wq, a, sms, s);
+  if (a.M <= 32) return launch_w8a8_fused_mp<32, F32>(x, ldx, wq, a, sms, s);
+  return launch_w8a8_fused_mp<64, F32>(x, ldx, wq, a, sms, s);
+}
+
 // Tile width of the channel-wise pair tiles (256 x BN): the persistent pairs run ceil(tiles / pairs)
 // rounds of work proportional to BN, plus a cost per tile that grows as tiles narrow (each tile
 // re-reads its 256 token rows from L2; measured: at M = 16384, N = 7168 tiles of 256 beat 224 by
@@ -388,6 +482,8 @@ static i8q_status launch_w8a8_any(const int8_t* xq, const int8_t* wq, const W8A8
   if (a.M <= 32) return launch_w8a8_small_mp<32, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
   if (a.M <= 64) return launch_w8a8_small_mp<64, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
   if (a.M <= W8A8_SMALL_MAX_M) return launch_w8a8_small_mp<128, BLOCKWISE, F32, DBG>(xq, wq, a, sms, s);
+  // output rows that are not 16-byte aligned take the element-wise epilogue (its own instantiation)
+  if (a.N % 8 != 0) return launch_w8a8<256, BLOCKWISE, F32, DBG, false>(xq, wq, a, sms, s);
   if constexpr (!BLOCKWISE) {
     switch (channel_tile_n(a.M, a.N, sms)) {
       case 224: return launch_w8a8<224, false, F32, DBG>(xq, wq, a, sms, s);
@@ -574,7 +670,7 @@ i8q_status i8q_gemm_w8a8_channel(const int8_t* xq, const float* sx, const int8_t
     if (dbg) I8Q_CUDA(cudaMemsetAsync(dbg, 0, (size_t)M * N * 4, S(stream)));
     return I8Q_OK;
   }
-  W8A8Args a{sx, 0, sw, (int)M, (int)N, (int)K, y, dbg};
+  W8A8Args a{sx, 0, sw, (int)M, (int)N, (int)K, y, dbg, nullptr, 1};
   if (dbg) return launch_w8a8_any<false, false, true>(xq, wq, a, sms, S(stream));
   return launch_w8a8_any<false, false, false>(xq, wq, a, sms, S(stream));
 }
@@ -594,7 +690,7 @@ i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx,
     I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * osz, S(stream)));
     return I8Q_OK;
   }
-  W8A8Args a{sx, ld_sx, sw, (int)M, (int)N, (int)K, y, dbg};
+  W8A8Args a{sx, ld_sx, sw, (int)M, (int)N, (int)K, y, dbg, nullptr, 1};
   const bool f32 = out == I8Q_OUT_FP32;
   if (dbg) {
     if (f32) return launch_w8a8_any<true, true, true>(xq, wq, a, sms, S(stream));
@@ -602,6 +698,82 @@ i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx,
   }
   if (f32) return launch_w8a8_any<true, true, false>(xq, wq, a, sms, S(stream));
   return launch_w8a8_any<true, false, false>(xq, wq, a, sms, S(stream));
+}
+
+// ---------------------------------------------------------------- a1 fused into a4 ----------
+i8q_status i8q_gemm_w8a8_block_fused_quant(const uint16_t* x, int64_t ldx, const int8_t* wq, const float* sw,
+                                           int64_t M, int64_t N, int64_t K, void* y, i8q_out_dtype out,
+                                           int8_t* xq_out, float* sx_out, int64_t ld_sx, void* stream) {
+  I8Q_REQUIRE(out == I8Q_OUT_BF16 || out == I8Q_OUT_FP32, I8Q_ERR_DTYPE);
+  I8Q_REQUIRE(M >= 0 && N >= 0 && K >= 0 && N < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(M <= kFusedQuantMaxM && K % 128 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(127LL * 127LL * K < (1LL << 31), I8Q_ERR_SHAPE);
+  if (M == 0 || N == 0) return I8Q_OK;
+  I8Q_REQUIRE(y, I8Q_ERR_NULL);
+  I8Q_REQUIRE(aligned16(y) && aligned16(xq_out) && aligned16(sx_out), I8Q_ERR_ALIGN);
+  if (sx_out) I8Q_REQUIRE(ld_sx >= M && ld_sx % 4 == 0, I8Q_ERR_SHAPE);
+  int sms;
+  i8q_status st = current_device(&sms);
+  if (st) return st;
+  const size_t osz = out == I8Q_OUT_FP32 ? 4 : 2;
+  if (K == 0) {
+    I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * osz, S(stream)));
+    return I8Q_OK;
+  }
+  I8Q_REQUIRE(x && wq && sw, I8Q_ERR_NULL);
+  I8Q_REQUIRE(ldx >= K && ldx % 8 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(aligned16(x) && aligned16(wq) && aligned16(sw), I8Q_ERR_ALIGN);
+  W8A8Args a{nullptr, ld_sx, sw, (int)M, (int)N, (int)K, y, nullptr, nullptr, 1, xq_out, sx_out};
+  if (out == I8Q_OUT_FP32) return launch_w8a8_fused<true>(x, ldx, wq, a, sms, S(stream));
+  return launch_w8a8_fused<false>(x, ldx, wq, a, sms, S(stream));
+}
+
+// ---------------------------------------------------------------- grouped (MoE) a5, a4 ------
+i8q_status i8q_gemm_w8a8_channel_grouped(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                                         const int32_t* expert_offsets, int64_t E, int64_t M, int64_t N, int64_t K,
+                                         uint16_t* y, int32_t* dbg, void* stream) {
+  i8q_status st = gemm_w8a8_common_checks(xq, sx, wq, sw, M, N, K, y, dbg);
+  if (st || M == 0 || N == 0) return st;
+  st = grouped_checks(expert_offsets, E, M, N, K);
+  if (st) return st;
+  int sms;
+  st = current_device(&sms);
+  if (st) return st;
+  if (K == 0) {
+    I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * 2, S(stream)));
+    if (dbg) I8Q_CUDA(cudaMemsetAsync(dbg, 0, (size_t)M * N * 4, S(stream)));
+    return I8Q_OK;
+  }
+  W8A8Args a{sx, 0, sw, (int)M, (int)N, (int)K, y, dbg, expert_offsets, (int)E};
+  if (dbg) return launch_w8a8_grouped<false, false, true>(xq, wq, a, sms, S(stream));
+  return launch_w8a8_grouped<false, false, false>(xq, wq, a, sms, S(stream));
+}
+
+i8q_status i8q_gemm_w8a8_block_grouped(const int8_t* xq, const float* sx, int64_t ld_sx, const int8_t* wq,
+                                       const float* sw, const int32_t* expert_offsets, int64_t E, int64_t M,
+                                       int64_t N, int64_t K, void* y, i8q_out_dtype out, int32_t* dbg, void* stream) {
+  I8Q_REQUIRE(out == I8Q_OUT_BF16 || out == I8Q_OUT_FP32, I8Q_ERR_DTYPE);
+  i8q_status st = gemm_w8a8_common_checks(xq, sx, wq, sw, M, N, K, y, dbg);
+  if (st || M == 0 || N == 0) return st;
+  if (K > 0) I8Q_REQUIRE(ld_sx >= M && ld_sx % 4 == 0, I8Q_ERR_SHAPE);
+  st = grouped_checks(expert_offsets, E, M, N, K);
+  if (st) return st;
+  int sms;
+  st = current_device(&sms);
+  if (st) return st;
+  const size_t osz = out == I8Q_OUT_FP32 ? 4 : 2;
+  if (K == 0) {
+    I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * osz, S(stream)));
+    return I8Q_OK;
+  }
+  W8A8Args a{sx, ld_sx, sw, (int)M, (int)N, (int)K, y, dbg, expert_offsets, (int)E};
+  const bool f32 = out == I8Q_OUT_FP32;
+  if (dbg) {
+    if (f32) return launch_w8a8_grouped<true, true, true>(xq, wq, a, sms, S(stream));
+    return launch_w8a8_grouped<true, false, true>(xq, wq, a, sms, S(stream));
+  }
+  if (f32) return launch_w8a8_grouped<true, true, false>(xq, wq, a, sms, S(stream));
+  return launch_w8a8_grouped<true, false, false>(xq, wq, a, sms, S(stream));
 }
 
 // ---------------------------------------------------------------- a6 -------------------------

@@ -47,6 +47,9 @@ _SIGS = {
     "i8q_gemm_w8a8_block": [_P, _P, _I, _P, _P, _I, _I, _I, _P, ctypes.c_int, _P, _P],
     "i8q_gemm_w8a8_channel": [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P],
     "i8q_gemm_w8a16_group": [_P, _P, _P, _I, _I, _I, _P, _P],
+    "i8q_gemm_w8a8_channel_grouped": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P],
+    "i8q_gemm_w8a8_block_fused_quant": [_P, _I, _P, _P, _I, _I, _I, _P, ctypes.c_int, _P, _P, _I, _P],
+    "i8q_gemm_w8a8_block_grouped": [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_int, _P, _P],
     "i8q_status_check": [_P],
     "i8q_test_set_wait_limit_ns": [ctypes.c_uint64],
     "i8q_test_skip_accumulator_signal": [ctypes.c_int],
@@ -153,12 +156,44 @@ def i8q_gemm_w8a8_block(xq, sx, wq, sw, y, out: int = I8Q_OUT_BF16, debug_partia
           M, N, K, _ptr(y), int(out), _ptr(debug_partials), _stream(stream))
 
 
+def i8q_gemm_w8a8_block_fused_quant(x, wq, sw, y, out: int = I8Q_OUT_BF16, xq_out=None, sx_out=None,
+                                    ld_sx: Optional[int] = None, stream=None) -> None:
+    """y [M, N] = block-wise W8A8 GEMM of bf16 x [M, K] (M <= 64) with the per-token-group
+    quantization done inside the GEMM; xq_out [M, K] / sx_out [K/128, ld_sx] optionally receive the
+    quantized activations."""
+    M, K = x.shape
+    N = wq.shape[0]
+    if ld_sx is None:
+        ld_sx = sx_out.shape[1] if sx_out is not None else 0
+    _call("i8q_gemm_w8a8_block_fused_quant", _ptr(x), _ld(x), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), int(out),
+          _ptr(xq_out), _ptr(sx_out), ld_sx, _stream(stream))
+
+
 def i8q_gemm_w8a8_channel(xq, sx, wq, sw, y, debug_acc=None, stream=None) -> None:
     """y [M, N] bf16 = channel-wise W8A8 GEMM with sx [M], sw [N]."""
     M, K = xq.shape
     N = wq.shape[0]
     _call("i8q_gemm_w8a8_channel", _ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), _ptr(debug_acc),
           _stream(stream))
+
+
+def i8q_gemm_w8a8_channel_grouped(xq, sx, wq, sw, expert_offsets, y, debug_acc=None, stream=None) -> None:
+    """Grouped (MoE) channel-wise GEMM: xq [M, K] sorted by expert, wq [E, N, K], sw [E, N],
+    expert_offsets int32 [E + 1] on the device, y [M, N] bf16."""
+    M, K = xq.shape
+    E, N = wq.shape[0], wq.shape[1]
+    _call("i8q_gemm_w8a8_channel_grouped", _ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(expert_offsets), E, M, N,
+          K, _ptr(y), _ptr(debug_acc), _stream(stream))
+
+
+def i8q_gemm_w8a8_block_grouped(xq, sx, wq, sw, expert_offsets, y, out: int = I8Q_OUT_BF16, debug_partials=None,
+                                ld_sx: Optional[int] = None, stream=None) -> None:
+    """Grouped (MoE) block-wise GEMM: xq [M, K] sorted by expert, sx [K/128, ld_sx], wq [E, N, K],
+    sw [E, ceil(N/128), K/128], expert_offsets int32 [E + 1] on the device, y [M, N]."""
+    M, K = xq.shape
+    E, N = wq.shape[0], wq.shape[1]
+    _call("i8q_gemm_w8a8_block_grouped", _ptr(xq), _ptr(sx), sx.shape[1] if ld_sx is None else ld_sx, _ptr(wq),
+          _ptr(sw), _ptr(expert_offsets), E, M, N, K, _ptr(y), int(out), _ptr(debug_partials), _stream(stream))
 
 
 def i8q_gemm_w8a16_group(x, wq, s, y, stream=None) -> None:

@@ -96,14 +96,15 @@ def activation_f16(M: int, K: int, seed: int, sigma: float = 1.0,
 
 
 def int8_weight_groups(N: int, K: int, seed: int, group: int = 128,
-                       sigma: float = 0.02, stream: int = STREAM_W):
+                       sigma: float = 0.02, stream: int = STREAM_W, scale_fmt: str = "fp16"):
     """A stored symmetric group-wise INT8 weight (W8A16 checkpoint format).
 
     Codes are drawn directly as integers: a rounded N(0, 42) clipped to
     +-127, with one entry per group forced to +-127 as a symmetric absmax
-    quantizer would leave it.  Group scales are fp16 values of
-    U(2.5*sigma, 4.5*sigma) / 127, i.e. the scale an absmax quantizer gives a
-    N(0, sigma) group.  Returns (wq int8 [N, K], s fp16 bits [N, K/group]).
+    quantizer would leave it.  Group scales are fp16 (or, with
+    scale_fmt="bf16", bf16) values of U(2.5*sigma, 4.5*sigma) / 127, i.e. the
+    scale an absmax quantizer gives a N(0, sigma) group.
+    Returns (wq int8 [N, K], s fp16 / bf16 bits [N, K/group]).
     """
     assert K % group == 0
     rng = _rng(seed, stream)
@@ -114,7 +115,12 @@ def int8_weight_groups(N: int, K: int, seed: int, group: int = 128,
     qv = q.reshape(N, g, group)
     qv[np.arange(N)[:, None], np.arange(g)[None, :], pos] = sign
     s = rng.uniform(2.5 * sigma, 4.5 * sigma, size=(N, g)).astype(np.float32) / np.float32(127.0)
-    return q, _f32_to_f16_bits(s)
+    return q, (_f32_to_bf16_bits(s) if scale_fmt == "bf16" else _f32_to_f16_bits(s))
+
+
+def activation_bf16_plain(M: int, K: int, seed: int, sigma: float = 1.0, stream: int = STREAM_X) -> np.ndarray:
+    """Activations X ~ N(0, sigma) without outliers (bf16 W8A16 inputs); bf16 bits [M, K]."""
+    return activation_bf16(M, K, seed, outlier_p=0.0, sigma=sigma, stream=stream)
 
 
 def token_counts(E: int, total: int, seed: int, stream: int = STREAM_X) -> np.ndarray:

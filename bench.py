@@ -141,6 +141,16 @@ def describe(name: str, args) -> dict:
                               f"W[{N},{K}] bf16 out; step = per-token-group act quant + INT8 GEMM",
                   "M": M, "N": N, "K": K, "global_batch": M * world, "seq_len": 1,
                   "parallelism": f"dp{world}", "l2": f"{R} rotating input/output copies (> 2x L2 per cycle)"}
+    elif name in ("moe_channel", "moe_block"):
+        E, N, K = 32, 7168, 2048
+        M = args.M or 8192
+        R = 2
+        scheme = "channel-wise" if name == "moe_channel" else "block-wise"
+        config = {"workload": f"grouped (MoE) {scheme} W8A8, DeepSeek-R1 MoE expert down-proj: {E} experts "
+                              f"W[{E},{N},{K}], {M} routed token rows X[{M},{K}] (ragged seeded counts) bf16 out; "
+                              f"step = act quant + grouped INT8 GEMM",
+                  "M": M, "N": N, "K": K, "experts": E, "global_batch": M * world, "seq_len": 1,
+                  "parallelism": f"dp{world}", "l2": "2 rotating activation/output copies; 470 MB of weights"}
     elif name == "requant":
         M, N, K, R = 0, 18432, 7168, 2
         config = {"workload": f"offline FP8-E4M3 [{N},{K}] (128x128 fp32 scales) -> BF16 -> INT8 128x128 block requant",
@@ -447,7 +457,115 @@ class W8A16(Workload):
         return [("gemm_w8a16_group", f"a6 W8A16 GEMM M={self.M} N={self.N} K={self.K}", "hbm", self.dom_bytes)]
 
 
-WORKLOADS = {"w8a8_channel": ChannelW8A8, "w8a8_block": BlockW8A8, "requant": Requant, "w8a16": W8A16}
+class GroupedW8A8(Workload):
+    """Grouped (MoE) W8A8 layer: 32 experts of the DeepSeek-R1 MoE down-proj shape, token rows
+    sorted by expert with seeded ragged counts (some experts may get none); per step the routed
+    rows are quantized and every expert's rows multiplied by that expert's weight."""
+    name = "moe_channel"
+
+    def __init__(self, args, rank=0):
+        super().__init__(args)
+        import torch
+        from activation_quantized_gemm_b200 import i8q, synth
+        self.q = i8q
+        self.block = args.workload == "moe_block"
+        self.name = args.workload
+        d = describe(args.workload, args)
+        E, M, N, K = d["config"]["experts"], d["M"], d["N"], d["K"]
+        self.E, self.M, self.N, self.K = E, M, N, K
+        KB = K // 128
+        counts = synth.token_counts(E, M, seed=6)
+        off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        x = synth.activation_bf16(M, K, seed=shard_seed(6, rank), outlier_p=0.001, outlier_mult=50.0)
+        dev = "cuda"
+        self.wq = torch.empty((E, N, K), dtype=torch.int8, device=dev)
+        self.sw = (torch.empty((E, (N + 127) // 128, KB), dtype=torch.float32, device=dev) if self.block
+                   else torch.empty((E, N), dtype=torch.float32, device=dev))
+        for e in range(E):                                       # offline weight quantization
+            wd = torch.from_numpy(synth.weight_bf16(N, K, seed=600 + e).view(np.int16)).to(dev)
+            if self.block:
+                i8q.i8q_quant_weight_block(wd, self.wq[e], self.sw[e])
+            else:
+                i8q.i8q_quant_act_token(wd, self.wq[e], self.sw[e])
+        self.off = torch.from_numpy(off).to(dev)
+        ld = (M + 3) // 4 * 4
+        self.R = 2
+        self.bufs = []
+        for r in range(self.R):
+            self.bufs.append({
+                "x": torch.from_numpy(x.view(np.int16)).to(dev),
+                "xq": torch.empty((M, K), dtype=torch.int8, device=dev),
+                "sx": (torch.empty((KB, ld), dtype=torch.float32, device=dev) if self.block
+                       else torch.empty((M,), dtype=torch.float32, device=dev)),
+                "y": torch.empty((M, N), dtype=torch.int16, device=dev)})
+        self.x_host = torch.from_numpy(x.view(np.int16)).pin_memory()
+        self.y_host = torch.empty((M, N), dtype=torch.int16).pin_memory()
+        qk = "quant_act_token_group" if self.block else "quant_act_token"
+        gk = "gemm_w8a8_block_grouped" if self.block else "gemm_w8a8_channel_grouped"
+        self.kernels = [qk, gk]
+        self.units_per_step = 2.0 * M * N * K / 1e12
+        self.dominant = gk
+        self.dom_units = self.units_per_step
+        self.dom_bound = "tensor"
+        self.dom_bytes = M * K + E * N * K + 2 * M * N
+        self.h2d_bytes = M * K * 2
+        self.d2h_bytes = M * N * 2
+        self.config = d["config"]
+
+    def launch(self, i, k, stream):
+        b = self.bufs[i % self.R]
+        if k == 0:
+            if self.block:
+                self.q.i8q_quant_act_token_group(b["x"], b["xq"], b["sx"], stream=stream)
+            else:
+                self.q.i8q_quant_act_token(b["x"], b["xq"], b["sx"], stream=stream)
+        elif self.block:
+            self.q.i8q_gemm_w8a8_block_grouped(b["xq"], b["sx"], self.wq, self.sw, self.off, b["y"], stream=stream)
+        else:
+            self.q.i8q_gemm_w8a8_channel_grouped(b["xq"], b["sx"], self.wq, self.sw, self.off, b["y"], stream=stream)
+
+    def e2e_step(self, i, stream):
+        b = self.bufs[i % self.R]
+        b["x"].copy_(self.x_host, non_blocking=True)
+        self.launch(i, 0, stream)
+        self.launch(i, 1, stream)
+        self.y_host.copy_(b["y"], non_blocking=True)
+
+    def oracle_sample(self, budget_s):
+        from oracle import ref_cpp as O
+        from activation_quantized_gemm_b200 import synth
+        E, N, K = self.E, self.N, self.K
+        counts = synth.token_counts(E, self.M, seed=6)
+        off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
+        e0 = int(np.argmax(counts))                              # a sample of one expert's rows
+        w = synth.weight_bf16(N, K, seed=600 + e0)
+        x = synth.activation_bf16(int(counts[e0]), K, seed=6, outlier_p=0.001, outlier_mult=50.0)
+        wq, sw = O.quant_weight_block(w) if self.block else O.quant_act_token(w)
+
+        def run(rows):
+            t0 = time.perf_counter()
+            if self.block:
+                xq, sx = O.quant_act_token_group(x[:rows])
+                O.gemm_w8a8_block_grouped(xq, sx, wq[None], sw[None], np.array([0, rows]))
+            else:
+                xq, sx = O.quant_act_token(x[:rows])
+                O.gemm_w8a8_channel_grouped(xq, sx, wq[None], sw[None], np.array([0, rows]))
+            return time.perf_counter() - t0
+        rows = _scale_rows(run, 1, x.shape[0], budget_s)
+        dt = run(rows)
+        return 2.0 * rows * N * K / 1e12, dt, f"{rows} token rows of expert {e0} (quant + GEMM), N={N}, K={K}"
+
+    def sub_results(self):
+        M, N, K = self.M, self.N, self.K
+        qk, gk = self.kernels
+        qbytes = 3 * M * K + (4 * M * (K // 128) if self.block else 4 * M)
+        return [(qk, f"act quant of the routed rows [{M},{K}]", "hbm", qbytes),
+                (gk, f"grouped {'block' if self.block else 'channel'}-wise GEMM, {self.E} experts, "
+                     f"M={M} N={N} K={K}", "tensor", self.dom_units * 1e12)]
+
+
+WORKLOADS = {"w8a8_channel": ChannelW8A8, "w8a8_block": BlockW8A8, "requant": Requant, "w8a16": W8A16,
+             "moe_channel": GroupedW8A8, "moe_block": GroupedW8A8}
 
 
 # ---------------------------------------------------------------------------------- clocks
@@ -567,6 +685,8 @@ SUB_WORKLOADS = [
     ("channel_m16", "w8a8_channel", 16, "up"),
     ("block_up_m16", "w8a8_block", 16, "up"),
     ("block_down_m16", "w8a8_block", 16, "down"),
+    ("moe_channel_e32", "moe_channel", 8192, "up"),
+    ("moe_block_e32", "moe_block", 8192, "up"),
     ("requant", "requant", 0, "up"),
     ("w8a16_m16_n12288", "w8a16", 16, "up"),
     ("w8a16_m16_n4096", "w8a16", 16, "down"),
@@ -728,6 +848,8 @@ def run_reference(args):
     cfg = d["config"]
     if args.workload == "w8a16":
         wl.units_per_step = (wl.N * wl.K + 2 * wl.N * (wl.K // 128) + 2 * wl.M * wl.K + 2 * wl.M * wl.N) / 1e9
+    if cls is GroupedW8A8:
+        wl.E, wl.block = cfg["experts"], args.workload == "moe_block"
     budget = max(0.5, min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         wl.oracle_sample(budget)

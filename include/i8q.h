@@ -138,6 +138,31 @@ i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx,
                                void* y, i8q_out_dtype out, int32_t* debug_partials, void* stream);
 
 /*
+ * Block-wise W8A8 GEMM with the online per-token-group activation quantization fused in
+ * (decode batches).  [R1-INT8] section 2.3, block-wise paragraph: the activations are quantized
+ * online per token-group of 128 and consumed by the INT8 matmul with a dequantization per K slab.
+ * The result is the composition i8q_quant_act_token_group followed by i8q_gemm_w8a8_block, and is
+ * bit-identical to it (the same quantizer code runs inside the GEMM, on the activation slab each
+ * CTA stages next to its weight slab), without the separate launch and the HBM round trip of the
+ * int8 activations.
+ *   x_bf16 : [M][ldx] bf16, K valid columns; ldx >= K, ldx % 8 == 0.
+ *   wq, sw : as i8q_gemm_w8a8_block ([N][K] int8, [ceil(N/128)][K/128] fp32).
+ *   1 <= M <= 64: decode batches only (I8Q_ERR_SHAPE above): for larger M every X slab would be
+ *   quantized again by each of the ceil(N/256) tiles that read it, which costs more than the
+ *   stand-alone quantizer; use i8q_quant_act_token_group + i8q_gemm_w8a8_block there.
+ *   N >= 0 (any N); K >= 0, K % 128 == 0.
+ *   y : [M][N] bf16 or fp32 (out).
+ *   xq_out, sx_out : NULL, or receive the quantized activations exactly as
+ *            i8q_quant_act_token_group writes them ([M][K] int8; [K/128][ld_sx] fp32,
+ *            ld_sx >= M, ld_sx % 4 == 0); ld_sx is ignored when sx_out is NULL.
+ * M == 0 or N == 0 is a no-op; K == 0 writes y = 0.
+ */
+i8q_status i8q_gemm_w8a8_block_fused_quant(const uint16_t* x_bf16, int64_t ldx, const int8_t* wq,
+                                           const float* sw, int64_t M, int64_t N, int64_t K, void* y,
+                                           i8q_out_dtype out, int8_t* xq_out, float* sx_out, int64_t ld_sx,
+                                           void* stream);
+
+/*
  * Channel-wise W8A8 GEMM: y[m][n] = bf16( float(A[m][n]) * (sx[m] * sw[n]) ),
  * A = xq wq^T accumulated exactly in int32.
  * [R1-INT8] section 2.3, channel-wise paragraph and Fig. 3 (right): a single dequantization
@@ -151,6 +176,36 @@ i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx,
 i8q_status i8q_gemm_w8a8_channel(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
                                  int64_t M, int64_t N, int64_t K,
                                  uint16_t* y_bf16, int32_t* debug_acc, void* stream);
+
+/*
+ * Grouped (MoE) W8A8 GEMMs: many experts, each with its own quantized weight and scales, over
+ * one batch of token rows sorted by expert.
+ * [R1-INT8] section 2.3 (the block-wise and channel-wise schemes above, applied per expert);
+ * [FP8-vs-INT8] section 3.1.2 (the MoE expert weights of DeepSeek models are quantized like the
+ * dense ones).  Row m of xq belongs to the expert e with off[e] <= m < off[e + 1]; its output row
+ * is the dense GEMM of that row with expert e's weight:
+ *   channel: y[m][n] = bf16( float(A) * (sx[m] * sw[e][n]) ),  A = sum_k xq[m][k] * wq[e][n][k];
+ *   block:   y[m][n] = sum_kb P * (sx[m][kb] * sw[e][n/128][kb]) in fp32, as i8q_gemm_w8a8_block.
+ *   xq  : [M][K] int8, rows sorted by expert.
+ *   sx  : channel [M] fp32; block [K/128][ld_sx] fp32 (token-contiguous, ld_sx >= M, % 4 == 0).
+ *   wq  : [E][N][K] int8 (the experts' weights stacked);  sw : channel [E][N]; block
+ *         [E][ceil(N/128)][K/128] fp32.
+ *   expert_offsets : DEVICE array of E + 1 int32, non-decreasing, off[0] = 0, off[E] = M (routing
+ *         is device data: the host need not know the per-expert counts; an expert may have none).
+ *         The kernel clamps the offsets to be non-decreasing within [0, M], so rows outside
+ *         [off[0], off[E]) are never written and no row outside [0, M) is ever touched.
+ *   1 <= E <= 1024; E * N < 2^31; N >= 0 (any N); K >= 0, K % 128 == 0; M >= 0.
+ *   y : [M][N] bf16 (channel) or bf16 / fp32 by `out` (block).
+ *   debug_acc / debug_partials : NULL or as in the dense calls ([M][N], [M][N][K/128]).
+ * M == 0 or N == 0 is a no-op; K == 0 writes y = 0.
+ */
+i8q_status i8q_gemm_w8a8_channel_grouped(const int8_t* xq, const float* sx, const int8_t* wq, const float* sw,
+                                         const int32_t* expert_offsets, int64_t E, int64_t M, int64_t N,
+                                         int64_t K, uint16_t* y_bf16, int32_t* debug_acc, void* stream);
+i8q_status i8q_gemm_w8a8_block_grouped(const int8_t* xq, const float* sx, int64_t ld_sx, const int8_t* wq,
+                                       const float* sw, const int32_t* expert_offsets, int64_t E, int64_t M,
+                                       int64_t N, int64_t K, void* y, i8q_out_dtype out,
+                                       int32_t* debug_partials, void* stream);
 
 /*
  * W8A16 group-wise weight-only GEMM (decode).
