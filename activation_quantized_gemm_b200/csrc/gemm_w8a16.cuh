@@ -1,7 +1,10 @@
-// W8A16 group-wise weight-only GEMM for decode batches (M <= 64), after
-// "DeepSeek-R1-0528-Qwen3-8B量化版发布" (technical details: symmetric group-wise INT8 Linear
-// weights, FP16 activations), group size 128 along K:
+// W8A16 group-wise weight-only GEMM, after "DeepSeek-R1-0528-Qwen3-8B量化版发布" (technical
+// details: symmetric group-wise INT8 Linear weights, FP16 activations), group size 128 along K:
 //     y[m][n] = fp16( sum_g s[n][g] * sum_{k in g} x[m][k] * wq[n][k] ).
+// BF16 = true: the same GEMM for a bf16 model (bf16 activations, group scales and output), the
+// weight-only INT8 analogue of the TensorRT-LLM build in "DeepSeek-R1-Distill-Llama-8B模型量化实战"
+// section 2.1.  Decode batches take one token tile of MP in {16, 32, 64} tokens (K split over a
+// cluster); larger batches (prefill) run tiles of 128 tokens, the grid's z dimension.
 //
 // The kernel streams the int8 weights once from HBM (the bound) and never rounds a dequantized
 // weight: int8 -> f16 is exact (|q| <= 127), the tensor core forms exact f16 x f16 products with
@@ -31,17 +34,18 @@
 // share of the rows over all ranks, in rank order, and writes fp16).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "common.cuh"
 
 namespace i8q {
 
-constexpr int W8A16_MAX_M = 64;
 constexpr int W8A16_BN = 128;   // weight rows per tile (MMA M)
 
 template <int MP>
 struct W8A16Cfg {
+  static_assert(MP == 16 || MP == 32 || MP == 64 || MP == 128, "token tile");
   static constexpr int W_BYTES = W8A16_BN * 128;         // int8 weight slab
   static constexpr int X_HALF = MP * 128;                // one 64-element half of the f16 slab
   static constexpr int X_BYTES = 2 * X_HALF;
@@ -51,8 +55,8 @@ struct W8A16Cfg {
   static constexpr int SLOT_COLS = A_COLS + MP;          // operand buffer + accumulator
   static constexpr int R_FIT = TMEM_COLS / SLOT_COLS;
   static constexpr int R = R_FIT < 4 ? R_FIT : 4;        // TMEM slots
-  static constexpr int W_STAGES = MP <= 16 ? 5 : (MP <= 32 ? 4 : 8);   // weight ring (freed after conversion)
-  static constexpr int X_STAGES = MP <= 16 ? 6 : 5;      // activation ring (freed by the MMA)
+  static constexpr int W_STAGES = MP <= 16 ? 5 : (MP <= 32 ? 4 : (MP <= 64 ? 8 : 4));   // weight ring (freed after conversion)
+  static constexpr int X_STAGES = MP <= 16 ? 6 : (MP <= 64 ? 5 : 4);   // activation ring (freed by the MMA)
   static constexpr int NUM_THREADS = 320;                // warps 0-3 epilogue, 4-7 converters, 8 TMA, 9 MMA
   static constexpr int RING_BYTES = W_STAGES * W_BYTES + X_STAGES * X_BYTES;
   static constexpr int SMEM_BYTES = RING_BYTES + 512 + 1024;
@@ -64,9 +68,9 @@ struct W8A16Cfg {
 };
 
 struct W8A16Args {
-  const uint16_t* s;   // [N][K/128] fp16 group scales
+  const uint16_t* s;   // [N][K/128] fp16 (bf16) group scales
   int M, N, K;
-  uint16_t* y;         // [M][N] fp16
+  uint16_t* y;         // [M][N] fp16 (bf16)
 };
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -118,6 +122,44 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// Instruction descriptor: kind::f16 with bf16 A and B, f32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4)               // D format: f32
+         | (1u << 7) | (1u << 10)  // A, B: bf16
+         | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// 4 signed int8 (one 32-bit word) -> 4 exact bf16 values as two bf16x2 words.  bf16 has 8
+// significant bits, so |q| <= 127 is exact but the f16 offset trick below does not fit: the
+// magnitude m = |q| (per byte: x ^ mask + (mask & 1), no carry between bytes) goes into the
+// mantissa of 128.0 (bf16 0x4300 | m = 128 + m, m < 128), 128 is subtracted (exact), and the sign
+// bit of q is put back.
+__device__ __forceinline__ void i8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t sg = w & 0x80808080u;
+  const uint32_t t = sg >> 7;                       // 1 in each negative byte
+  const uint32_t mag = (w ^ (t * 0xFFu)) + t;       // per-byte |q|
+  const uint32_t a = __byte_perm(mag, 0x43434343u, 0x4140);
+  const uint32_t b = __byte_perm(mag, 0x43434343u, 0x4342);
+  const __nv_bfloat162 c128 = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)0x4300),
+                                                 __ushort_as_bfloat16((unsigned short)0x4300));
+  __nv_bfloat162 ha = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&a), c128);
+  __nv_bfloat162 hb = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&b), c128);
+  lo = *reinterpret_cast<uint32_t*>(&ha) | __byte_perm(sg, 0u, 0x1404);
+  hi = *reinterpret_cast<uint32_t*>(&hb) | __byte_perm(sg, 0u, 0x3424);
+}
+
+// Group scale (fp16 or bf16 bits) -> fp32 (exact), and fp32 -> output bits (round to nearest even).
+template <bool BF16>
+__device__ __forceinline__ float half_bits_to_f32(uint16_t h) {
+  if constexpr (BF16) return __uint_as_float((uint32_t)h << 16);
+  else return __half2float(__ushort_as_half(h));
+}
+template <bool BF16>
+__device__ __forceinline__ uint16_t f32_to_half_bits(float v) {
+  if constexpr (BF16) return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  else return __half_as_ushort(__float2half_rn(v));
+}
+
 // 4 signed int8 (one 32-bit word) -> 4 exact f16 values as two half2 words.
 // Byte u = q + 128 is placed in the mantissa of 1024 (f16 0x6400); subtracting 1152 = 1024 + 128
 // leaves q exactly.
@@ -132,7 +174,7 @@ __device__ __forceinline__ void i8x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t
   hi = *reinterpret_cast<uint32_t*>(&hb);
 }
 
-template <int MP>
+template <int MP, bool BF16>
 __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
     k_gemm_w8a16(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                  const W8A16Args args) {
@@ -159,6 +201,7 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
   const int kb0 = (int)((int64_t)KB * rank / nrank), kb1 = (int)((int64_t)KB * (rank + 1) / nrank);
   const int nslab = kb1 - kb0;
   const int n0 = blockIdx.x * W8A16_BN;
+  const int m0 = blockIdx.z * MP;              // first token of this CTA's token tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::W_STAGES; ++s) {
@@ -218,8 +261,8 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
         } else {
           uint8_t* xs = sX + st * C::X_BYTES;
           mbar_arrive_expect_tx(&fullb[st], C::X_BYTES);
-          tma_load_2d(xs, &tmX, &fullb[st], kk, 0);
-          tma_load_2d(xs + C::X_HALF, &tmX, &fullb[st], kk + 64, 0);
+          tma_load_2d(xs, &tmX, &fullb[st], kk, m0);
+          tma_load_2d(xs + C::X_HALF, &tmX, &fullb[st], kk + 64, m0);
         }
         filled |= 1u << st;
         par = (par & ~(1u << st)) | (ph << st);
@@ -230,7 +273,7 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
     }
   } else if (warp == 9) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16(W8A16_BN, MP);
+      constexpr uint32_t idesc = BF16 ? idesc_bf16(W8A16_BN, MP) : idesc_f16(W8A16_BN, MP);
       for (int j = 0; j < nslab; ++j) {
         const int xs = j % C::X_STAGES;
         const int r = j % R;
@@ -272,10 +315,17 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint4 v = *reinterpret_cast<const uint4*>(wrow + (((4 * h + i) ^ sw) << 4));
-          i8x4_to_f16x4(v.x, o[8 * i + 0], o[8 * i + 1]);
-          i8x4_to_f16x4(v.y, o[8 * i + 2], o[8 * i + 3]);
-          i8x4_to_f16x4(v.z, o[8 * i + 4], o[8 * i + 5]);
-          i8x4_to_f16x4(v.w, o[8 * i + 6], o[8 * i + 7]);
+          if constexpr (BF16) {
+            i8x4_to_bf16x4(v.x, o[8 * i + 0], o[8 * i + 1]);
+            i8x4_to_bf16x4(v.y, o[8 * i + 2], o[8 * i + 3]);
+            i8x4_to_bf16x4(v.z, o[8 * i + 4], o[8 * i + 5]);
+            i8x4_to_bf16x4(v.w, o[8 * i + 6], o[8 * i + 7]);
+          } else {
+            i8x4_to_f16x4(v.x, o[8 * i + 0], o[8 * i + 1]);
+            i8x4_to_f16x4(v.y, o[8 * i + 2], o[8 * i + 3]);
+            i8x4_to_f16x4(v.z, o[8 * i + 4], o[8 * i + 5]);
+            i8x4_to_f16x4(v.w, o[8 * i + 6], o[8 * i + 7]);
+          }
         }
         tmem_st32(tmem + lane_addr + r * C::A_COLS + h * 32, o);
       }
@@ -307,11 +357,11 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
       __syncwarp();
     };
     for (int r = 0; r < R; ++r) free_slot(r);   // every accumulator starts out free
-    float sc_next = (n < N && nslab > 0) ? __half2float(__ushort_as_half(__ldg(args.s + (int64_t)n * G + kb0))) : 0.f;
+    float sc_next = (n < N && nslab > 0) ? half_bits_to_f32<BF16>(__ldg(args.s + (int64_t)n * G + kb0)) : 0.f;
     for (int j = 0; j < nslab; ++j) {
       const int r = j % R;
       const float sc = sc_next;
-      if (j + 1 < nslab && n < N) sc_next = __half2float(__ushort_as_half(__ldg(args.s + (int64_t)n * G + kb0 + j + 1)));
+      if (j + 1 < nslab && n < N) sc_next = half_bits_to_f32<BF16>(__ldg(args.s + (int64_t)n * G + kb0 + j + 1));
       if (!warp_wait(&mdone[r], (j / R) & 1, SITE_TMEM_FULL, abort_flag)) break;
       tc_fence_after();
       const uint32_t base = tmem + lane_addr + R * C::A_COLS + r * MP;
@@ -334,14 +384,15 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
   // its block of rows over all ranks, in rank order, 4 tokens per 16-byte load.
   tc_fence_before();
   __syncthreads();
-  const int mlim = args.M < MP ? args.M : MP;
+  const int mlim = args.M - m0 < MP ? args.M - m0 : MP;   // tokens of this tile
+  uint16_t* ytile = args.y + (int64_t)m0 * N;
   if (nrank == 1) {
     if (warp < 4) {
       const int n = n0 + warp * 32 + lane;
       if (n < N) {
 #pragma unroll
         for (int m = 0; m < MP; ++m)
-          if (m < mlim) args.y[(int64_t)m * N + n] = __half_as_ushort(__float2half_rn(sum[m]));
+          if (m < mlim) ytile[(int64_t)m * N + n] = f32_to_half_bits<BF16>(sum[m]);
       }
     }
   } else {
@@ -377,7 +428,7 @@ __global__ void __launch_bounds__(320, W8A16Cfg<MP>::CTAS_PER_SM)
         const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          if (4 * m4 + k < mlim) args.y[(int64_t)(4 * m4 + k) * N + n] = __half_as_ushort(__float2half_rn(vv[k]));
+          if (4 * m4 + k < mlim) ytile[(int64_t)(4 * m4 + k) * N + n] = f32_to_half_bits<BF16>(vv[k]);
       }
     }
   }

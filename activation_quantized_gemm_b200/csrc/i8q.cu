@@ -240,23 +240,25 @@ static int w8a8_small_splits(int64_t tiles, int64_t KB, int sms, int cps) {
   return s;
 }
 
-template <int MP>
+template <int MP, bool BF16>
 static i8q_status launch_w8a16_mp(const uint16_t* x, const int8_t* wq, const uint16_t* s, int M, int N, int K,
                                   uint16_t* y, int sms, cudaStream_t stream) {
   using C = W8A16Cfg<MP>;
-  auto kern = k_gemm_w8a16<MP>;
+  auto kern = k_gemm_w8a16<MP, BF16>;
   const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
   if (attr) return attr;
   CUtensorMap tw, tx;
   i8q_status st = make_tmap_2d(&tw, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, W8A16_BN, 128,
                                CU_TENSOR_MAP_SWIZZLE_128B);
   if (st) return st;
-  st = make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, K, K, MP, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  st = make_tmap_2d(&tx, x, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, M, K, K,
+                    MP, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (st) return st;
   const int64_t tiles = cdiv(N, W8A16_BN);
-  const int splits = decode_splits(tiles, K / 128, sms, C::CTAS_PER_SM);
+  const int64_t mtiles = cdiv(M, MP);           // token tiles (one for decode batches)
+  const int splits = decode_splits(tiles * mtiles, K / 128, sms, C::CTAS_PER_SM);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits, 1);
+  cfg.gridDim = dim3((unsigned)tiles, (unsigned)splits, (unsigned)mtiles);
   cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
@@ -274,11 +276,13 @@ static i8q_status launch_w8a16_mp(const uint16_t* x, const int8_t* wq, const uin
   return I8Q_OK;
 }
 
+template <bool BF16>
 static i8q_status launch_w8a16(const uint16_t* x, const int8_t* wq, const uint16_t* s, int M, int N, int K,
                                uint16_t* y, int sms, cudaStream_t stream) {
-  if (M <= 16) return launch_w8a16_mp<16>(x, wq, s, M, N, K, y, sms, stream);
-  if (M <= 32) return launch_w8a16_mp<32>(x, wq, s, M, N, K, y, sms, stream);
-  return launch_w8a16_mp<64>(x, wq, s, M, N, K, y, sms, stream);
+  if (M <= 16) return launch_w8a16_mp<16, BF16>(x, wq, s, M, N, K, y, sms, stream);
+  if (M <= 32) return launch_w8a16_mp<32, BF16>(x, wq, s, M, N, K, y, sms, stream);
+  if (M <= 64) return launch_w8a16_mp<64, BF16>(x, wq, s, M, N, K, y, sms, stream);
+  return launch_w8a16_mp<128, BF16>(x, wq, s, M, N, K, y, sms, stream);   // prefill: 128-token tiles
 }
 
 // ------------------------------------------------------------------ W8A8 launch -------------
@@ -777,10 +781,10 @@ i8q_status i8q_gemm_w8a8_block_grouped(const int8_t* xq, const float* sx, int64_
 }
 
 // ---------------------------------------------------------------- a6 -------------------------
-i8q_status i8q_gemm_w8a16_group(const uint16_t* x, const int8_t* wq, const uint16_t* s, int64_t M, int64_t N,
-                                int64_t K, uint16_t* y, void* stream) {
-  I8Q_REQUIRE(M >= 0 && N >= 0 && K >= 0 && N < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
-  I8Q_REQUIRE(M <= W8A16_MAX_M && K % 128 == 0, I8Q_ERR_SHAPE);
+static i8q_status gemm_w8a16_any(const uint16_t* x, const int8_t* wq, const uint16_t* s, int64_t M, int64_t N,
+                                 int64_t K, uint16_t* y, bool bf16, void* stream) {
+  I8Q_REQUIRE(M >= 0 && N >= 0 && K >= 0 && M < kMaxDim && N < kMaxDim && K < kMaxDim, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(cdiv(M, 128) < 65536 && K % 128 == 0, I8Q_ERR_SHAPE);   // token tiles: the grid's z dimension
   if (M == 0 || N == 0) return I8Q_OK;
   I8Q_REQUIRE(y, I8Q_ERR_NULL);
   I8Q_REQUIRE(aligned16(y), I8Q_ERR_ALIGN);
@@ -793,7 +797,18 @@ i8q_status i8q_gemm_w8a16_group(const uint16_t* x, const int8_t* wq, const uint1
   }
   I8Q_REQUIRE(x && wq && s, I8Q_ERR_NULL);
   I8Q_REQUIRE(aligned16(x) && aligned16(wq) && aligned16(s), I8Q_ERR_ALIGN);
-  return launch_w8a16(x, wq, s, (int)M, (int)N, (int)K, y, sms, S(stream));
+  if (bf16) return launch_w8a16<true>(x, wq, s, (int)M, (int)N, (int)K, y, sms, S(stream));
+  return launch_w8a16<false>(x, wq, s, (int)M, (int)N, (int)K, y, sms, S(stream));
+}
+
+i8q_status i8q_gemm_w8a16_group(const uint16_t* x, const int8_t* wq, const uint16_t* s, int64_t M, int64_t N,
+                                int64_t K, uint16_t* y, void* stream) {
+  return gemm_w8a16_any(x, wq, s, M, N, K, y, false, stream);
+}
+
+i8q_status i8q_gemm_w8a16_group_bf16(const uint16_t* x, const int8_t* wq, const uint16_t* s, int64_t M, int64_t N,
+                                     int64_t K, uint16_t* y, void* stream) {
+  return gemm_w8a16_any(x, wq, s, M, N, K, y, true, stream);
 }
 
 }  // extern "C"

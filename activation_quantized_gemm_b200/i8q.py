@@ -47,6 +47,7 @@ _SIGS = {
     "i8q_gemm_w8a8_block": [_P, _P, _I, _P, _P, _I, _I, _I, _P, ctypes.c_int, _P, _P],
     "i8q_gemm_w8a8_channel": [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P],
     "i8q_gemm_w8a16_group": [_P, _P, _P, _I, _I, _I, _P, _P],
+    "i8q_gemm_w8a16_group_bf16": [_P, _P, _P, _I, _I, _I, _P, _P],
     "i8q_gemm_w8a8_channel_grouped": [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P],
     "i8q_gemm_w8a8_block_fused_quant": [_P, _I, _P, _P, _I, _I, _I, _P, ctypes.c_int, _P, _P, _I, _P],
     "i8q_gemm_w8a8_block_grouped": [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_int, _P, _P],
@@ -201,6 +202,13 @@ def i8q_gemm_w8a16_group(x, wq, s, y, stream=None) -> None:
     M, K = x.shape
     N = wq.shape[0]
     _call("i8q_gemm_w8a16_group", _ptr(x), _ptr(wq), _ptr(s), M, N, K, _ptr(y), _stream(stream))
+
+
+def i8q_gemm_w8a16_group_bf16(x, wq, s, y, stream=None) -> None:
+    """y [M, N] bf16 = W8A16 group-wise GEMM; x [M, K] bf16, wq [N, K] int8, s [N, K/128] bf16."""
+    M, K = x.shape
+    N = wq.shape[0]
+    _call("i8q_gemm_w8a16_group_bf16", _ptr(x), _ptr(wq), _ptr(s), M, N, K, _ptr(y), _stream(stream))
 
 
 def i8q_status_check(stream=None) -> None:

@@ -155,13 +155,23 @@ def describe(name: str, args) -> dict:
         M, N, K, R = 0, 18432, 7168, 2
         config = {"workload": f"offline FP8-E4M3 [{N},{K}] (128x128 fp32 scales) -> BF16 -> INT8 128x128 block requant",
                   "N": N, "K": K, "parallelism": f"dp{world}", "l2": "2 rotating copies of 264 MB"}
-    elif name == "w8a16":
+    elif name in ("w8a16", "w8a16_bf16"):
         M = args.M or 16
         N, K = (12288, 4096) if args.proj == "up" else (4096, 12288)
         R = _rotations(N * K + 2 * N * (K // 128) + 2 * M * K + 2 * M * N)
-        config = {"workload": f"W8A16 group-128 decode GEMM, Qwen3-8B linear X fp16[{M},{K}] W int8[{N},{K}]",
-                  "M": M, "N": N, "K": K, "global_batch": M * world, "parallelism": f"dp{world}",
-                  "l2": f"{R} rotating copies (> 2x L2 per cycle)"}
+        dt = "bf16" if name == "w8a16_bf16" else "fp16"
+        kind = "decode" if M <= 64 else "prefill"
+        config = {"workload": f"W8A16 group-128 {kind} GEMM, Qwen3-8B linear X {dt}[{M},{K}] W int8[{N},{K}] "
+                              f"{dt} out", "M": M, "N": N, "K": K, "global_batch": M * world,
+                  "parallelism": f"dp{world}", "l2": f"{R} rotating copies (> 2x L2 per cycle)"}
+    elif name == "w8a8_block_fused":
+        N, K = (18432, 7168) if args.proj == "up" else (7168, 18432)
+        M = args.M or 16
+        R = _rotations(M * K * 2 + N * K + 2 * M * N)
+        config = {"workload": f"block-wise W8A8 decode linear, DeepSeek-R1 dense MLP {args.proj}-proj X[{M},{K}] "
+                              f"W[{N},{K}] bf16 out; step = one GEMM with the per-token-group act quant fused in",
+                  "M": M, "N": N, "K": K, "global_batch": M * world, "seq_len": 1,
+                  "parallelism": f"dp{world}", "l2": f"{R} rotating input/output copies (> 2x L2 per cycle)"}
     else:
         raise ValueError(name)
     return {"M": M, "N": N, "K": K, "R": R, "config": config}
@@ -394,6 +404,8 @@ class Requant(Workload):
 
 
 class W8A16(Workload):
+    """W8A16 group-wise GEMM (Qwen3-8B linear shapes): fp16 or bf16 activations; decode batches are
+    HBM-bound (GB/s), prefill batches (M > 256) tensor-bound against the 16-bit dense peak."""
     name = "w8a16"
     unit = "GB/s"
 
@@ -402,11 +414,17 @@ class W8A16(Workload):
         import torch
         from activation_quantized_gemm_b200 import i8q, synth
         self.q = i8q
+        self.bf16 = args.workload == "w8a16_bf16"
+        self.name = args.workload
         M = args.M or 16
         N, K = (12288, 4096) if args.proj == "up" else (4096, 12288)
         self.M, self.N, self.K = M, N, K
-        x = synth.activation_f16(M, K, seed=shard_seed(4, rank))
-        wq, s = synth.int8_weight_groups(N, K, seed=4)
+        if self.bf16:
+            x = synth.activation_bf16_plain(M, K, seed=shard_seed(4, rank))
+            wq, s = synth.int8_weight_groups(N, K, seed=4, scale_fmt="bf16")
+        else:
+            x = synth.activation_f16(M, K, seed=shard_seed(4, rank))
+            wq, s = synth.int8_weight_groups(N, K, seed=4)
         per_copy = N * K + 2 * N * (K // 128) + 2 * M * K + 2 * M * N
         self.R = _rotations(per_copy)
         dev = "cuda"
@@ -418,19 +436,28 @@ class W8A16(Workload):
                 "y": torch.empty((M, N), dtype=torch.int16, device=dev)})
         self.x_host = torch.from_numpy(x.view(np.int16)).pin_memory()
         self.y_host = torch.empty((M, N), dtype=torch.int16).pin_memory()
-        self.kernels = ["gemm_w8a16_group"]
-        self.units_per_step = per_copy / 1e9
-        self.dominant = "gemm_w8a16_group"
-        self.dom_units = per_copy / 1e9
-        self.dom_bound = "hbm"
+        self.kernels = ["gemm_w8a16_group_bf16" if self.bf16 else "gemm_w8a16_group"]
+        self.dominant = self.kernels[0]
         self.dom_bytes = per_copy
+        if M > 256:                       # prefill: tensor-bound, TFLOP/s of the 16-bit MMAs
+            self.unit = "TFLOP/s"
+            self.units_per_step = 2.0 * M * N * K / 1e12
+            self.dom_units = self.units_per_step
+            self.dom_bound = "tensor16"
+        else:
+            self.units_per_step = per_copy / 1e9
+            self.dom_units = per_copy / 1e9
+            self.dom_bound = "hbm"
         self.h2d_bytes = 2 * M * K
         self.d2h_bytes = 2 * M * N
         self.config = describe(self.name, args)["config"]
 
     def launch(self, i, k, stream):
         b = self.bufs[i % self.R]
-        self.q.i8q_gemm_w8a16_group(b["x"], b["wq"], b["s"], b["y"], stream=stream)
+        if self.bf16:
+            self.q.i8q_gemm_w8a16_group_bf16(b["x"], b["wq"], b["s"], b["y"], stream=stream)
+        else:
+            self.q.i8q_gemm_w8a16_group(b["x"], b["wq"], b["s"], b["y"], stream=stream)
 
     def e2e_step(self, i, stream):
         b = self.bufs[i % self.R]
@@ -441,20 +468,105 @@ class W8A16(Workload):
     def oracle_sample(self, budget_s):
         from oracle import ref_cpp as O
         from activation_quantized_gemm_b200 import synth
-        x = synth.activation_f16(self.M, self.K, seed=4)
-        wq, s = synth.int8_weight_groups(self.N, self.K, seed=4)
+        bf16 = getattr(self, "bf16", False)
+        Ms = min(self.M, 64)
+        if bf16:
+            x = synth.activation_bf16_plain(Ms, self.K, seed=4)
+            wq, s = synth.int8_weight_groups(self.N, self.K, seed=4, scale_fmt="bf16")
+        else:
+            x = synth.activation_f16(Ms, self.K, seed=4)
+            wq, s = synth.int8_weight_groups(self.N, self.K, seed=4)
 
         def run(rows):                       # rows of W (output channels)
             t0 = time.perf_counter()
-            O.gemm_w8a16_group(x, wq[:rows], s[:rows])
+            O.gemm_w8a16_group_fmt(x, wq[:rows], s[:rows], "bf16" if bf16 else "fp16")
             return time.perf_counter() - t0
         rows = _scale_rows(run, 64, self.N, budget_s)
         dt = run(rows)
-        frac = rows / self.N
-        return self.units_per_step * frac, dt, f"{rows} of {self.N} weight rows, M={self.M}, K={self.K}"
+        frac = rows / self.N * Ms / self.M
+        return self.units_per_step * frac, dt, (f"{rows} of {self.N} weight rows x {Ms} of {self.M} tokens, "
+                                                f"K={self.K}")
 
     def sub_results(self):
-        return [("gemm_w8a16_group", f"a6 W8A16 GEMM M={self.M} N={self.N} K={self.K}", "hbm", self.dom_bytes)]
+        dt = "bf16" if self.bf16 else "fp16"
+        units = self.dom_units * 1e12 if self.dom_bound == "tensor16" else self.dom_bytes
+        return [(self.kernels[0], f"a6 W8A16 GEMM ({dt}) M={self.M} N={self.N} K={self.K}", self.dom_bound, units)]
+
+
+class FusedBlockW8A8(Workload):
+    """Block-wise decode layer with the activation quantization inside the GEMM (one launch per
+    step, i8q_gemm_w8a8_block_fused_quant); compare its step with the two-launch block workload."""
+    name = "w8a8_block_fused"
+    unit = "GB/s"
+
+    def __init__(self, args, rank=0):
+        super().__init__(args)
+        import torch
+        from activation_quantized_gemm_b200 import i8q, synth
+        self.q = i8q
+        d = describe(self.name, args)
+        M, N, K = d["M"], d["N"], d["K"]
+        self.M, self.N, self.K = M, N, K
+        x = synth.activation_bf16(M, K, seed=shard_seed(2, rank), outlier_p=0.001, outlier_mult=50.0)
+        w = synth.weight_bf16(N, K, seed=2)
+        dev = "cuda"
+        wd = torch.from_numpy(w.view(np.int16)).to(dev)
+        self.R = d["R"]
+        self.bufs = []
+        for r in range(self.R):
+            b = {"x": torch.from_numpy(x.view(np.int16)).to(dev),
+                 "wq": torch.empty((N, K), dtype=torch.int8, device=dev),
+                 "sw": torch.empty(((N + 127) // 128, K // 128), dtype=torch.float32, device=dev),
+                 "y": torch.empty((M, N), dtype=torch.int16, device=dev)}
+            i8q.i8q_quant_weight_block(wd, b["wq"], b["sw"])
+            self.bufs.append(b)
+        del wd
+        self.x_host = torch.from_numpy(x.view(np.int16)).pin_memory()
+        self.y_host = torch.empty((M, N), dtype=torch.int16).pin_memory()
+        self.kernels = ["gemm_w8a8_block_fused_quant"]
+        self.dom_bytes = 2 * M * K + N * K + 4 * ((N + 127) // 128) * (K // 128) + 2 * M * N
+        self.units_per_step = self.dom_bytes / 1e9
+        self.dominant = self.kernels[0]
+        self.dom_units = self.units_per_step
+        self.dom_bound = "hbm"
+        self.h2d_bytes = M * K * 2
+        self.d2h_bytes = M * N * 2
+        self.config = d["config"]
+
+    def launch(self, i, k, stream):
+        b = self.bufs[i % self.R]
+        self.q.i8q_gemm_w8a8_block_fused_quant(b["x"], b["wq"], b["sw"], b["y"], stream=stream)
+
+    def e2e_step(self, i, stream):
+        b = self.bufs[i % self.R]
+        b["x"].copy_(self.x_host, non_blocking=True)
+        self.launch(i, 0, stream)
+        self.y_host.copy_(b["y"], non_blocking=True)
+
+    def oracle_sample(self, budget_s):
+        """The oracle's a1 then a4 for all M tokens on a subset of the weight rows; units are the
+        step's bytes scaled by the fraction of the output computed."""
+        from oracle import ref_cpp as O
+        from activation_quantized_gemm_b200 import synth
+        w = synth.weight_bf16(self.N, self.K, seed=2)
+        wq, sw = O.quant_weight_block(w)                           # offline, not timed
+        x = synth.activation_bf16(self.M, self.K, seed=2, outlier_p=0.001, outlier_mult=50.0)
+
+        def run(rows):
+            rows = -(-rows // 128) * 128
+            t0 = time.perf_counter()
+            xq, sx = O.quant_act_token_group(x)
+            O.gemm_w8a8_block(xq, sx, wq[:rows], sw[: rows // 128])
+            return time.perf_counter() - t0
+        rows = _scale_rows(run, 128, self.N, budget_s)
+        rows = min(self.N, -(-rows // 128) * 128)
+        dt = run(rows)
+        step_bytes = 2 * self.M * self.K + self.N * self.K + 2 * self.M * self.N
+        return step_bytes * rows / self.N / 1e9, dt, f"{rows} of {self.N} weight rows, all {self.M} tokens (a1 + a4)"
+
+    def sub_results(self):
+        return [(self.kernels[0], f"a1 fused into a4, block-wise GEMM {self.args.proj}-proj M={self.M} "
+                                  f"N={self.N} K={self.K}", "hbm", self.dom_bytes)]
 
 
 class GroupedW8A8(Workload):
@@ -565,7 +677,8 @@ class GroupedW8A8(Workload):
 
 
 WORKLOADS = {"w8a8_channel": ChannelW8A8, "w8a8_block": BlockW8A8, "requant": Requant, "w8a16": W8A16,
-             "moe_channel": GroupedW8A8, "moe_block": GroupedW8A8}
+             "w8a16_bf16": W8A16, "moe_channel": GroupedW8A8, "moe_block": GroupedW8A8,
+             "w8a8_block_fused": FusedBlockW8A8}
 
 
 # ---------------------------------------------------------------------------------- clocks
@@ -669,11 +782,14 @@ def _measure(wl, steps: int, warmup: int, hold_ms: float, stream, barrier, clock
 
 def _figure(bound: str, units: float, ms: float, peaks) -> dict:
     """Throughput of `units` (ops for a tensor-bound kernel, bytes otherwise) in `ms`, and its
-    fraction of the measured peak."""
+    fraction of the measured peak (INT8 for "tensor", 16-bit for "tensor16", HBM copy otherwise)."""
     if bound == "tensor":
         v = units / 1e12 / (ms / 1e3)
         peak = peaks["bf16_tflops"] * INT8_PER_BF16
         return {"value": round(v, 2), "unit": "TOPS", "frac": round(v / peak, 4)}
+    if bound == "tensor16":
+        v = units / 1e12 / (ms / 1e3)
+        return {"value": round(v, 2), "unit": "TFLOP/s", "frac": round(v / peaks["bf16_tflops"], 4)}
     v = units / 1e9 / (ms / 1e3)
     return {"value": round(v, 1), "unit": "GB/s", "frac": round(v / peaks["hbm_gbs"], 4)}
 
@@ -685,11 +801,16 @@ SUB_WORKLOADS = [
     ("channel_m16", "w8a8_channel", 16, "up"),
     ("block_up_m16", "w8a8_block", 16, "up"),
     ("block_down_m16", "w8a8_block", 16, "down"),
+    ("block_up_m16_fused", "w8a8_block_fused", 16, "up"),
+    ("block_down_m16_fused", "w8a8_block_fused", 16, "down"),
     ("moe_channel_e32", "moe_channel", 8192, "up"),
     ("moe_block_e32", "moe_block", 8192, "up"),
     ("requant", "requant", 0, "up"),
     ("w8a16_m16_n12288", "w8a16", 16, "up"),
     ("w8a16_m16_n4096", "w8a16", 16, "down"),
+    ("w8a16_bf16_m16_n12288", "w8a16_bf16", 16, "up"),
+    ("w8a16_prefill_m2048_n12288", "w8a16", 2048, "up"),
+    ("w8a16_bf16_prefill_m2048_n12288", "w8a16_bf16", 2048, "up"),
 ]
 
 
@@ -789,6 +910,11 @@ def run_ours(args):
             achieved = wl.dom_units / (dom_ms / 1e3)
             unit = "TOPS"
             peak_note = f"INT8 dense = {src} burst bf16 {peaks['bf16_tflops']} TFLOP/s x {INT8_PER_BF16} (nominal ratio)"
+        elif wl.dom_bound == "tensor16":
+            peak = peaks["bf16_tflops"]
+            achieved = wl.dom_units / (dom_ms / 1e3)
+            unit = "TFLOP/s"
+            peak_note = f"{src} burst bf16 dense (fp16 the same rate)"
         else:
             peak = peaks["hbm_gbs"]
             achieved = wl.dom_bytes / 1e9 / (dom_ms / 1e3)
@@ -846,8 +972,13 @@ def run_reference(args):
     d = describe(args.workload, args)
     wl.M, wl.N, wl.K = d["M"], d["N"], d["K"]
     cfg = d["config"]
-    if args.workload == "w8a16":
-        wl.units_per_step = (wl.N * wl.K + 2 * wl.N * (wl.K // 128) + 2 * wl.M * wl.K + 2 * wl.M * wl.N) / 1e9
+    if cls is W8A16:
+        wl.bf16 = args.workload == "w8a16_bf16"
+        if wl.M > 256:
+            wl.unit = "TFLOP/s"
+            wl.units_per_step = 2.0 * wl.M * wl.N * wl.K / 1e12
+        else:
+            wl.units_per_step = (wl.N * wl.K + 2 * wl.N * (wl.K // 128) + 2 * wl.M * wl.K + 2 * wl.M * wl.N) / 1e9
     if cls is GroupedW8A8:
         wl.E, wl.block = cfg["experts"], args.workload == "moe_block"
     budget = max(0.5, min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup)))

@@ -208,18 +208,30 @@ i8q_status i8q_gemm_w8a8_block_grouped(const int8_t* xq, const float* sx, int64_
                                        int32_t* debug_partials, void* stream);
 
 /*
- * W8A16 group-wise weight-only GEMM (decode).
+ * W8A16 group-wise weight-only GEMM.
  * [Qwen3-8B-W8A16], technical details: Linear weights are symmetric group-wise INT8, the
  * activations stay FP16.  Group size 128 along K:
- *   y[m][n] = fp16( sum_g s[n][g] * sum_{k in group g} x[m][k] * wq[n][k] )
- * with the products exact in fp32 and fp32 accumulation.
+ *   y[m][n] = fp16( sum_g s[n][g] * sum_{k in g} x[m][k] * wq[n][k] )
+ * with the products exact in fp32 and fp32 accumulation (the dequantized weight is never rounded).
  *   x_f16 : [M][K] fp16;  wq : [N][K] int8;  s_f16 : [N][K/128] fp16 group scales.
- *   1 <= M <= 64 (decode batch); N >= 0 (any N); K >= 0, K % 128 == 0.
+ *   M >= 0 (decode batches of up to 64 tokens run one token tile with K split over a cluster;
+ *   larger batches run 128-token tiles, ceil(M / 128) < 65536); N >= 0 (any N);
+ *   K >= 0, K % 128 == 0.
  *   y_f16 : [M][N] fp16 output (round to nearest even).
- * M == 0 or N == 0 is a no-op; K == 0 writes y = 0; M > 64 gives I8Q_ERR_SHAPE.
+ * M == 0 or N == 0 is a no-op; K == 0 writes y = 0.
  */
 i8q_status i8q_gemm_w8a16_group(const uint16_t* x_f16, const int8_t* wq, const uint16_t* s_f16,
                                 int64_t M, int64_t N, int64_t K, uint16_t* y_f16, void* stream);
+
+/*
+ * The same W8A16 group-wise GEMM for a BF16 model: bf16 activations, bf16 group scales, bf16
+ * output (round to nearest even).  The weight-only INT8 path of "DeepSeek-R1-Distill-Llama-8B
+ * 模型量化实战" section 2.1 (TensorRT-LLM, weights INT8, activations kept in 16-bit) with the group
+ * scales of [Qwen3-8B-W8A16].  int8 -> bf16 is exact (|q| <= 127 needs 7 bits); products are
+ * exact in fp32.  Arguments, layouts and limits as i8q_gemm_w8a16_group.
+ */
+i8q_status i8q_gemm_w8a16_group_bf16(const uint16_t* x_bf16, const int8_t* wq, const uint16_t* s_bf16,
+                                     int64_t M, int64_t N, int64_t K, uint16_t* y_bf16, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* i8q_status_string(i8q_status status);

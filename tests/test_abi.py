@@ -53,8 +53,8 @@ def test_shape_checks(lib):
     assert _st(lib, "i8q_quant_act_token_group", P, 3, 256, 256, P, P, 3, None) == 2
     # K so large that int32 accumulation could overflow
     assert _st(lib, "i8q_gemm_w8a8_channel", P, P, P, P, 4, 8, 133248, P, None, None) == 2
-    # W8A16 decode batch limit
-    assert _st(lib, "i8q_gemm_w8a16_group", P, P, P, 65, 128, 128, P, None) == 2
+    # W8A16: K not a multiple of 128
+    assert _st(lib, "i8q_gemm_w8a16_group_bf16", P, P, P, 65, 128, 100, P, None) == 2
 
 
 def test_null_align_dtype_checks(lib):

@@ -178,3 +178,30 @@ def test_w8a16_qwen3_8b(q, N, K):
         ms, ns = _grid(M, N, 8, 256, seed=N + M)
         Y, T = O.gemm_w8a16_group_at(x, wq, s, ms, ns)
         check_half(host(y, np.uint16)[ms, ns], Y, T, "fp16", f"w8a16 {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("N,K", [(12288, 4096), (4096, 12288)])
+def test_w8a16_qwen3_8b_prefill_and_bf16(q, N, K):
+    """Qwen3-8B shapes at prefill batches (fp16) and with bf16 activations (decode and prefill)."""
+    wq, s = synth.int8_weight_groups(N, K, seed=4)
+    wqd, sd = dev(wq), dev(s)
+    x_all = synth.activation_f16(2048, K, seed=4)
+    for M in [512, 2048]:
+        x = x_all[:M]
+        y = empty((M, N), torch.int16, 0x7E00)
+        q.i8q_gemm_w8a16_group(dev(x), wqd, sd, y)
+        torch.cuda.synchronize()
+        ms, ns = _grid(M, N, 16, 128, seed=N + M)
+        Y, T = O.gemm_w8a16_group_at(x, wq, s, ms, ns)
+        check_half(host(y, np.uint16)[ms, ns], Y, T, "fp16", f"w8a16 prefill {M}x{N}x{K}")
+    wqb, sb = synth.int8_weight_groups(N, K, seed=5, scale_fmt="bf16")
+    wqbd, sbd = dev(wqb), dev(sb)
+    xb_all = synth.activation_bf16_plain(2048, K, seed=5)
+    for M in [1, 16, 64, 2048]:
+        x = xb_all[:M]
+        y = empty((M, N), torch.int16, 0x7FC0)
+        q.i8q_gemm_w8a16_group_bf16(dev(x), wqbd, sbd, y)
+        torch.cuda.synchronize()
+        ms, ns = _grid(M, N, 16, 128, seed=N + M + 1)
+        Y, T = O.gemm_w8a16_group_at(x, wqb, sb, ms, ns, fmt="bf16")
+        check_half(host(y, np.uint16)[ms, ns], Y, T, "bf16", f"w8a16 bf16 {M}x{N}x{K}")
