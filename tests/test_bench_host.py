@@ -86,3 +86,36 @@ def test_traffic_sources_exist():
     for key, (traffic, src) in bench.MEASURED_TRAFFIC.items():
         assert traffic > 0, key
         assert os.path.exists(os.path.join(root, "profiles", src)), (key, src)
+
+
+def test_gpus_flag_spawns_one_process_per_gpu(monkeypatch):
+    """`bench.py --gpus N` without torchrun spawns N ranks itself, each with the rank environment
+    torchrun would give it (loopback rendezvous); under torchrun (WORLD_SIZE set) it spawns nothing."""
+    import sys
+    import torch.multiprocessing as mp
+    calls, envs = [], []
+
+    def fake_spawn(fn, args=(), nprocs=1, join=True):
+        calls.append(nprocs)
+        for r in range(nprocs):
+            fn(r, *args)
+
+    def fake_run(args):
+        import os
+        envs.append({k: os.environ[k] for k in ("RANK", "LOCAL_RANK", "WORLD_SIZE", "MASTER_ADDR", "MASTER_PORT")})
+
+    monkeypatch.setattr(mp, "spawn", fake_spawn)
+    monkeypatch.setattr(bench, "run_ours", fake_run)
+    for k in ("RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):   # restored after the test
+        monkeypatch.setenv(k, "x")
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "3"])
+    bench.main()
+    assert calls == [3]
+    assert [e["RANK"] for e in envs] == ["0", "1", "2"] and all(e["WORLD_SIZE"] == "3" for e in envs)
+    assert all(e["MASTER_ADDR"] == "127.0.0.1" and e["LOCAL_RANK"] == e["RANK"] for e in envs)
+    calls.clear()
+    envs.clear()
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.main()
+    assert calls == [] and len(envs) == 1
