@@ -47,9 +47,11 @@ struct W8A8SmallCfg {
   // fused: the bf16 activation slab has its own ring, freed as soon as the quantizers have read it
   static constexpr int XB_HALF = MP * 128;                // one 64-column half of the bf16 slab
   static constexpr int XB_BYTES = 2 * XB_HALF;
-  static constexpr int XR = FUSEDQ ? 2 : 0;               // bf16 ring stages
+  // bf16 ring stages: deep enough that an activation slab's L2 latency (~1 us) stays hidden
+  // behind the quantization of the slabs before it (two stages left the quantizers waiting)
+  static constexpr int XR = FUSEDQ ? (MP == 32 ? 3 : 4) : 0;   // (3 at 32 tokens: shared memory)
   static constexpr int XRING_BYTES = XR * XB_BYTES;
-  static constexpr int QW = FUSEDQ ? (MP <= 32 ? 1 : 2) : 0;   // quantizer warps
+  static constexpr int QW = FUSEDQ ? 2 : 0;               // quantizer warps
   static constexpr int NBUF = BLOCKWISE ? 4 : 1;          // slab accumulators in TMEM
   static constexpr int TMEM_NEED = NBUF * MP;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;

@@ -716,6 +716,11 @@ i8q_status i8q_gemm_w8a8_block_fused_quant(const uint16_t* x, int64_t ldx, const
   I8Q_REQUIRE(y, I8Q_ERR_NULL);
   I8Q_REQUIRE(aligned16(y) && aligned16(xq_out) && aligned16(sx_out), I8Q_ERR_ALIGN);
   if (sx_out) I8Q_REQUIRE(ld_sx >= M && ld_sx % 4 == 0, I8Q_ERR_SHAPE);
+  if (K > 0) {
+    I8Q_REQUIRE(x && wq && sw, I8Q_ERR_NULL);
+    I8Q_REQUIRE(ldx >= K && ldx % 8 == 0, I8Q_ERR_SHAPE);
+    I8Q_REQUIRE(aligned16(x) && aligned16(wq) && aligned16(sw), I8Q_ERR_ALIGN);
+  }
   int sms;
   i8q_status st = current_device(&sms);
   if (st) return st;
@@ -724,9 +729,6 @@ i8q_status i8q_gemm_w8a8_block_fused_quant(const uint16_t* x, int64_t ldx, const
     I8Q_CUDA(cudaMemsetAsync(y, 0, (size_t)M * N * osz, S(stream)));
     return I8Q_OK;
   }
-  I8Q_REQUIRE(x && wq && sw, I8Q_ERR_NULL);
-  I8Q_REQUIRE(ldx >= K && ldx % 8 == 0, I8Q_ERR_SHAPE);
-  I8Q_REQUIRE(aligned16(x) && aligned16(wq) && aligned16(sw), I8Q_ERR_ALIGN);
   W8A8Args a{nullptr, ld_sx, sw, (int)M, (int)N, (int)K, y, nullptr, nullptr, 1, xq_out, sx_out};
   if (out == I8Q_OUT_FP32) return launch_w8a8_fused<true>(x, ldx, wq, a, sms, S(stream));
   return launch_w8a8_fused<false>(x, ldx, wq, a, sms, S(stream));

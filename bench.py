@@ -735,8 +735,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------- main
 
 def _measure(wl, steps: int, warmup: int, hold_ms: float, stream, barrier, clocks=None):
-    """W warm-up steps, K timed steps back to back, then K steps with an event pair around every
-    launch.  Returns (total_ms of the back-to-back region, per-kernel mean launch ms)."""
+    """W warm-up steps, K timed steps back to back, then, for each kernel of the step, K launches of
+    that kernel alone back to back between one event pair.  Returns (total_ms of the back-to-back
+    step region, per-kernel mean launch ms).  (An event pair around every single launch would add
+    about 5 us of event overhead to each: an empty kernel measures 6 us that way.)"""
     import torch
     from activation_quantized_gemm_b200 import i8q
     nk = len(wl.kernels)
@@ -745,7 +747,6 @@ def _measure(wl, steps: int, warmup: int, hold_ms: float, stream, barrier, clock
             wl.launch(i, k, stream)
     i8q.i8q_status_check()
     barrier()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(steps)]
     if clocks is not None:
         clocks.start()
         time.sleep(0.3)
@@ -763,20 +764,23 @@ def _measure(wl, steps: int, warmup: int, hold_ms: float, stream, barrier, clock
             wl.launch(i, k, stream)
     t_end.record(stream)
     barrier()
-    # Per-kernel durations: the same K steps again with an event pair around every launch (the
-    # events keep each kernel from overlapping its neighbours, so these are whole launch durations).
-    torch.cuda._sleep(int(hold_ms * 1.9e6))
-    for i in range(steps):
-        ev[i][0].record(stream)
-        for k in range(nk):
+    # Per-kernel durations: each kernel of the step on its own, K launches back to back (the inputs
+    # of a later kernel are the outputs the earlier kernels left in the same rotating buffers).
+    per_kernel_ms = []
+    for k in range(nk):
+        k0 = torch.cuda.Event(enable_timing=True)
+        k1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(hold_ms * 1.9e6))
+        k0.record(stream)
+        for i in range(steps):
             wl.launch(i, k, stream)
-            ev[i][k + 1].record(stream)
-    barrier()
+        k1.record(stream)
+        barrier()
+        per_kernel_ms.append(k0.elapsed_time(k1) / steps)
     if clocks is not None:
         clocks.stop()
     i8q.i8q_status_check()
     total_ms = t_start.elapsed_time(t_end)
-    per_kernel_ms = [sum(ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(steps)) / steps for k in range(nk)]
     return total_ms, per_kernel_ms
 
 
@@ -947,9 +951,10 @@ def run_ours(args):
             line["sub_results"] = subs
             line["sub_results_note"] = (
                 "each entry timed in this run after the headline (its own warm-up and "
-                f"{args.sub_steps} steps, rotating >2x L2 of inputs); us = mean per-launch event time; "
-                "frac = of the measured HBM copy peak or the INT8 dense peak (bf16 burst x 2); "
-                "step_us = back-to-back step (launches overlap through programmatic dependent launch)")
+                f"{args.sub_steps} steps, rotating >2x L2 of inputs); us = mean launch time of that kernel "
+                "alone, back to back between one event pair; frac = of the measured HBM copy peak, the "
+                "INT8 dense peak (bf16 burst x 2) or the bf16 peak; step_us = back-to-back step of all its "
+                "kernels (launches overlap through programmatic dependent launch)")
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

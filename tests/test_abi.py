@@ -57,6 +57,24 @@ def test_shape_checks(lib):
     assert _st(lib, "i8q_gemm_w8a16_group_bf16", P, P, P, 65, 128, 100, P, None) == 2
 
 
+def test_new_entry_point_checks(lib):
+    # grouped: E out of range, offsets missing or misaligned
+    assert _st(lib, "i8q_gemm_w8a8_channel_grouped", P, P, P, P, P, 0, 4, 8, 128, P, None, None) == 2
+    assert _st(lib, "i8q_gemm_w8a8_channel_grouped", P, P, P, P, P, 1025, 4, 8, 128, P, None, None) == 2
+    assert _st(lib, "i8q_gemm_w8a8_channel_grouped", P, P, P, P, None, 4, 4, 8, 128, P, None, None) == 1
+    assert _st(lib, "i8q_gemm_w8a8_block_grouped", P, P, 4, P, P, U, 4, 4, 8, 128, P, 0, None, None) == 3
+    assert _st(lib, "i8q_gemm_w8a8_block_grouped", P, P, 4, P, P, P, 4, 4, 8, 128, P, 9, None, None) == 4
+    # fused quantization: decode batches only, K % 128, ldx >= K
+    assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", P, 128, P, P, 65, 8, 128, P, 0, None, None, 0, None) == 2
+    assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", P, 200, P, P, 4, 8, 200, P, 0, None, None, 0, None) == 2
+    assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", P, 64, P, P, 4, 8, 128, P, 0, None, None, 0, None) == 2
+    assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", P, 128, P, P, 4, 8, 128, P, 0, None, P, 2, None) == 2
+    # empty problems need no pointers
+    assert _st(lib, "i8q_gemm_w8a8_channel_grouped", None, None, None, None, None, 4, 0, 8, 128, None, None, None) == 0
+    assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", None, 0, None, None, 0, 8, 128, None, 0, None, None, 0, None) == 0
+    assert _st(lib, "i8q_gemm_w8a16_group_bf16", None, None, None, 0, 8, 128, None, None) == 0
+
+
 def test_null_align_dtype_checks(lib):
     assert _st(lib, "i8q_quant_act_token_group", None, 4, 128, 128, P, P, 4, None) == 1
     assert _st(lib, "i8q_gemm_w8a8_channel", P, None, P, P, 4, 8, 128, P, None, None) == 1

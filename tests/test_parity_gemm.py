@@ -27,7 +27,9 @@ SHAPES = [(1, 8, 128), (16, 256, 512), (7, 200, 384), (130, 264, 1024), (300, 52
           # any N: masked tails (unaligned output rows, a partial last weight block), decode and
           # prefill kernels
           (1, 1, 128), (16, 7, 256), (40, 129, 512), (300, 7, 384), (257, 129, 256), (33, 7170, 512),
-          (260, 7170, 256)]
+          (260, 7170, 256),
+          # M >= 512: several pair-tile rows, ragged last tile
+          (512, 1032, 1024), (600, 520, 768), (777, 7170, 512), (1024, 136, 2048)]
 
 
 @pytest.fixture(scope="module")
