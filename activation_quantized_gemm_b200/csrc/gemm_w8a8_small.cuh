@@ -17,7 +17,7 @@
 // Two CTAs share an SM for up to 64 tokens (rings of 4..6 stages each), one CTA for 128 (TMEM and
 // registers); the launch keeps all CTAs in one wave.
 //
-// FUSEDQ (block-wise, up to 64 tokens): the activations arrive as bf16 and are quantized inside
+// FUSEDQ (block-wise, up to 16 tokens): the activations arrive as bf16 and are quantized inside
 // the GEMM, per token and 128-wide K group, as "DeepSeek R1 INT8 quantization practice on SGLang"
 // section 2.3 prescribes ("quantized online per token-group").  The TMA warp stages the bf16 slab
 // [MP x 128] next to the weight slab; quantizer warps turn it into the int8 operand (128B-swizzled,
@@ -49,9 +49,15 @@ struct W8A8SmallCfg {
   static constexpr int XB_BYTES = 2 * XB_HALF;
   // bf16 ring stages: deep enough that an activation slab's L2 latency (~1 us) stays hidden
   // behind the quantization of the slabs before it (two stages left the quantizers waiting)
-  static constexpr int XR = FUSEDQ ? (MP == 32 ? 3 : 4) : 0;   // (3 at 32 tokens: shared memory)
+  // Quantizer warps.  Quantizing one slab is one long dependent chain for a warp (≈ 2000 cycles at
+  // 16 tokens, measured, more than a slab's share of the weight stream), so four warps take whole
+  // slabs in turn: warp q quantizes slabs j ≡ q mod 4 and owns the bf16 ring slots r ≡ q mod 4.
+  // Two slots per warp keep the next slab's bf16 load (≈ 1 µs from L2 under the weight stream)
+  // in flight while the warp quantizes the current one.
+  static constexpr int QW = FUSEDQ ? 4 : 0;
+  static constexpr int XR = FUSEDQ ? 2 * QW : 0;          // bf16 ring stages
   static constexpr int XRING_BYTES = XR * XB_BYTES;
-  static constexpr int QW = FUSEDQ ? 2 : 0;               // quantizer warps
+  static constexpr bool QALT = FUSEDQ;
   static constexpr int NBUF = BLOCKWISE ? 4 : 1;          // slab accumulators in TMEM
   static constexpr int TMEM_NEED = NBUF * MP;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : TMEM_NEED <= 256 ? 256 : 512;
@@ -76,9 +82,11 @@ struct W8A8SmallCfg {
   static_assert(STAGES >= 4, "stage ring");
   static_assert(MP * 128 * 4 <= STAGES * STAGE_BYTES, "reduction tile must fit in the stage buffers");
   static_assert(CPS * (SMEM_BYTES + CTA_RESERVED) <= SM_SMEM && SMEM_BYTES <= CTA_MAX, "shared memory");
-  static_assert(!FUSEDQ || (BLOCKWISE && MP <= 64), "fused quantization: block-wise, up to 64 tokens");
+  static_assert(!FUSEDQ || (BLOCKWISE && MP == 16), "fused quantization: block-wise, up to 16 tokens");
   static_assert(STAGE_BYTES % 1024 == 0, "128B-swizzled buffers stay 1024-byte aligned");
   static_assert(QR >= STAGES + NBUF, "scale ring deeper than the lead of the quantizer over the epilogue");
+  static_assert(8 * (3 * STAGES + 2 * NBUF + 1 + 2 * XR + (FUSEDQ ? QR : 0)) + 8 <= BAR_BYTES, "barrier block");
+  static_assert(!QALT || (XR % (QW > 0 ? QW : 1) == 0 && QW <= STAGES), "each bf16 slot belongs to one quantizer warp");
 };
 
 // Fused quantizer: quantize the bf16 activation slab of one stage (two 128B-swizzled halves of
@@ -158,8 +166,13 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS, FUSEDQ>::NUM_
   uint64_t* done = tempty + C::NBUF;
   uint64_t* xfull = done + 1;                 // fused: bf16 activation slab landed (ring of XR)
   uint64_t* xempty = xfull + C::XR;           // fused: bf16 slab read by the quantizers
-  uint64_t* qready = xempty + C::XR;          // fused: int8 operand and scales of the stage written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(FUSEDQ ? qready + C::STAGES : done + 1);
+  uint64_t* qready = xempty + C::XR;          // fused: int8 operand of the stage written
+  // fused: token scales of a slab written (ring of QR, the depth of the scale ring).  The epilogue
+  // cannot wait on qready: the quantizers may finish slab j + STAGES before the epilogue asks for
+  // slab j, and a parity wait cannot tell those two phases apart.  They cannot lap this ring (slab
+  // j + QR needs the epilogue past slab j, as QR >= STAGES + NBUF).
+  uint64_t* sready = qready + C::STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(FUSEDQ ? sready + C::QR : done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* qsx = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES + C::RING_BYTES);
 
@@ -189,9 +202,10 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS, FUSEDQ>::NUM_
     if constexpr (FUSEDQ) {
       for (int r = 0; r < C::XR; ++r) {
         mbar_init(&xfull[r], 1);
-        mbar_init(&xempty[r], C::QW);
+        mbar_init(&xempty[r], C::QALT ? 1 : C::QW);
       }
-      for (int st = 0; st < C::STAGES; ++st) mbar_init(&qready[st], C::QW);
+      for (int st = 0; st < C::STAGES; ++st) mbar_init(&qready[st], C::QALT ? 1 : C::QW);
+      for (int q = 0; q < C::QR; ++q) mbar_init(&sready[q], C::QALT ? 1 : C::QW);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -299,20 +313,23 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS, FUSEDQ>::NUM_
     // quantizers: bf16 activation slab -> int8 operand + per-token group scales (see quantize_slab)
     if constexpr (FUSEDQ) {
       const int qi = warp - (EW + 2);
-      for (int j = 0; j < nslab; ++j) {
+      // ALT: this warp's slabs are qi, qi + QW, ... (whole slabs); otherwise every slab, its tokens
+      for (int j = C::QALT ? qi : 0; j < nslab; j += C::QALT ? C::QW : 1) {
         const int s = j % C::STAGES, r = j % C::XR;
         if (!warp_wait(&xfull[r], (j / C::XR) & 1, SITE_FULL, abort_flag)) break;
         // the int8 operand buffer of stage s is free once the MMAs of slab j - STAGES are done
         if (!warp_wait(&empty[s], ((j / C::STAGES) & 1) ^ 1, SITE_EMPTY, abort_flag)) break;
-        quantize_slab<MP, C::QW>(xring + r * C::XB_BYTES, smem + s * C::STAGE_BYTES + C::W_BYTES,
-                                 qsx + (j % C::QR) * MP, qi, lane, blockIdx.x == 0 ? args.qx_out : nullptr,
-                                 blockIdx.x == 0 ? args.qs_out : nullptr, M, K, kb0 + j, args.ld_sx);
+        quantize_slab<MP, C::QALT ? 1 : C::QW>(xring + r * C::XB_BYTES, smem + s * C::STAGE_BYTES + C::W_BYTES,
+                                               qsx + (j % C::QR) * MP, C::QALT ? 0 : qi, lane,
+                                               blockIdx.x == 0 ? args.qx_out : nullptr,
+                                               blockIdx.x == 0 ? args.qs_out : nullptr, M, K, kb0 + j, args.ld_sx);
         // generic-proxy reads and writes of shared memory before the tensor core and TMA touch it
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&xempty[r]);
           mbar_arrive(&qready[s]);
+          mbar_arrive(&sready[j % C::QR]);
         }
       }
     }
@@ -360,7 +377,7 @@ __global__ void __launch_bounds__(W8A8SmallCfg<MP, BLOCKWISE, CPS, FUSEDQ>::NUM_
         float* slot = ring + (j & 1) * MPW;
         if constexpr (FUSEDQ) {
           // token scales of slab j come from the quantizer warps through shared memory
-          if (!warp_wait(&qready[j % C::STAGES], (j / C::STAGES) & 1, SITE_CONVERT, abort_flag)) break;
+          if (!warp_wait(&sready[j % C::QR], (j / C::QR) & 1, SITE_CONVERT, abort_flag)) break;
 #pragma unroll
           for (int i = 0; i < PER_LANE; ++i) {
             const int m = cb + lane + 32 * i;

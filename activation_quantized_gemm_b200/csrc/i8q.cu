@@ -180,7 +180,7 @@ static i8q_status ensure_smem(Kern k, int bytes) {
 }
 
 static constexpr int64_t kMaxDim = (int64_t)1 << 30;
-static constexpr int64_t kFusedQuantMaxM = 64;   // decode batches (see i8q_gemm_w8a8_block_fused_quant)
+static constexpr int64_t kFusedQuantMaxM = 16;   // decode batches (see i8q_gemm_w8a8_block_fused_quant)
 
 // Resident CTAs per SM of a kernel at a block size (queried once per kernel and block size).
 template <typename Kern>
@@ -418,12 +418,12 @@ static i8q_status launch_w8a8_small_mp(const int8_t* xq, const int8_t* wq, const
   return I8Q_OK;
 }
 
-// Block-wise GEMM with the activation quantization fused in (decode batches, M <= 64): the decode
+// Block-wise GEMM with the activation quantization fused in (decode batches, M <= 16): the decode
 // kernel with quantizer warps; X arrives as bf16 through its own TMA map.
 template <int MP, bool F32>
 static i8q_status launch_w8a8_fused_mp(const uint16_t* x, int64_t ldx, const int8_t* wq, const W8A8Args& a, int sms,
                                        cudaStream_t s) {
-  constexpr int CPS = MP <= 32 ? 2 : 1;
+  constexpr int CPS = 2;
   using C = W8A8SmallCfg<MP, true, CPS, true>;
   auto kern = k_gemm_w8a8_small<MP, true, CPS, F32, false, true>;
   const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
@@ -457,9 +457,7 @@ static i8q_status launch_w8a8_fused_mp(const uint16_t* x, int64_t ldx, const int
 template <bool F32>
 static i8q_status launch_w8a8_fused(const uint16_t* x, int64_t ldx, const int8_t* wq, const W8A8Args& a, int sms,
                                     cudaStream_t s) {
-  if (a.M <= 16) return launch_w8a8_fused_mp<16, F32>(x, ldx, wq, a, sms, s);
-  if (a.M <= 32) return launch_w8a8_fused_mp<32, F32>(x, ldx, wq, a, sms, s);
-  return launch_w8a8_fused_mp<64, F32>(x, ldx, wq, a, sms, s);
+  return launch_w8a8_fused_mp<16, F32>(x, ldx, wq, a, sms, s);
 }
 
 // Tile width of the channel-wise pair tiles (256 x BN): the persistent pairs run ceil(tiles / pairs)
@@ -616,6 +614,7 @@ i8q_status i8q_quant_act_token(const uint16_t* x, int64_t M, int64_t K, int64_t 
 // ---------------------------------------------------------------- a3', a3 --------------------
 i8q_status i8q_quant_weight_block(const uint16_t* w, int64_t N, int64_t K, int8_t* wq, float* sw, void* stream) {
   I8Q_REQUIRE(N >= 0 && K >= 0 && N < kMaxDim && K < kMaxDim && K % 128 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(cdiv(N, 128) * (K / 128) < kMaxDim, I8Q_ERR_SHAPE);   // block indices are 32-bit
   if (N == 0 || K == 0) return I8Q_OK;
   I8Q_REQUIRE(w && wq && sw, I8Q_ERR_NULL);
   I8Q_REQUIRE(aligned16(w) && aligned16(wq) && aligned16(sw), I8Q_ERR_ALIGN);

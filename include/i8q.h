@@ -86,7 +86,7 @@ i8q_status i8q_quant_act_token(const uint16_t* x_bf16, int64_t M, int64_t K, int
 /*
  * Block-wise 128x128 weight quantization of a BF16 weight.
  * [R1-INT8] section 2.3, block-wise paragraph (quantization within 128x128 blocks).
- *   w_bf16 : [N][K] bf16;  N >= 0;  K >= 0, K % 128 == 0.
+ *   w_bf16 : [N][K] bf16;  N >= 0;  K >= 0, K % 128 == 0;  ceil(N/128) * K/128 < 2^30 blocks.
  *   wq     : [N][K] int8 output.
  *   sw     : [ceil(N/128)][K/128] fp32 output; a partial last row-block takes the absmax over
  *            the rows present.
@@ -100,8 +100,8 @@ i8q_status i8q_quant_weight_block(const uint16_t* w_bf16, int64_t N, int64_t K,
  * per 128x128 block and no BF16 weights, so the weights are dequantized to BF16 first
  * (bf16 = round_to_nearest_even(fp32(e4m3) * sf), one fp32 multiply) and then block-quantized.
  * E4M3 is the OCP "E4M3FN" encoding (no infinities; NaN codes are outside the contract).
- *   w_e4m3 : [N][K] bytes;   sf : [ceil(N/128)][K/128] fp32 block scales of the FP8 tensor.
- *   N >= 0;  K >= 0, K % 128 == 0.
+ *   w_e4m3 : [N][K] bytes;   sf : [ceil(N/128)][K/128] finite fp32 block scales of the FP8 tensor.
+ *   N >= 0;  K >= 0, K % 128 == 0;  ceil(N/128) * K/128 < 2^30 blocks (I8Q_ERR_SHAPE otherwise).
  *   wq     : [N][K] int8 output;   sw : [ceil(N/128)][K/128] fp32 output.
  */
 i8q_status i8q_requant_fp8_to_int8_block(const uint8_t* w_e4m3, const float* sf, int64_t N, int64_t K,
@@ -147,9 +147,10 @@ i8q_status i8q_gemm_w8a8_block(const int8_t* xq, const float* sx, int64_t ld_sx,
  * int8 activations.
  *   x_bf16 : [M][ldx] bf16, K valid columns; ldx >= K, ldx % 8 == 0.
  *   wq, sw : as i8q_gemm_w8a8_block ([N][K] int8, [ceil(N/128)][K/128] fp32).
- *   1 <= M <= 64: decode batches only (I8Q_ERR_SHAPE above): for larger M every X slab would be
- *   quantized again by each of the ceil(N/256) tiles that read it, which costs more than the
- *   stand-alone quantizer; use i8q_quant_act_token_group + i8q_gemm_w8a8_block there.
+ *   1 <= M <= 16: decode batches only (I8Q_ERR_SHAPE above).  Every N tile quantizes the
+ *   activation slabs it reads, so the in-GEMM work grows with M: up to 16 tokens it is hidden
+ *   behind the weight stream (measured, DeepSeek-R1 up-projection), beyond that the separate
+ *   quantizer is cheaper; use i8q_quant_act_token_group + i8q_gemm_w8a8_block there.
  *   N >= 0 (any N); K >= 0, K % 128 == 0.
  *   y : [M][N] bf16 or fp32 (out).
  *   xq_out, sx_out : NULL, or receive the quantized activations exactly as

@@ -65,7 +65,7 @@ def test_new_entry_point_checks(lib):
     assert _st(lib, "i8q_gemm_w8a8_block_grouped", P, P, 4, P, P, U, 4, 4, 8, 128, P, 0, None, None) == 3
     assert _st(lib, "i8q_gemm_w8a8_block_grouped", P, P, 4, P, P, P, 4, 4, 8, 128, P, 9, None, None) == 4
     # fused quantization: decode batches only, K % 128, ldx >= K
-    assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", P, 128, P, P, 65, 8, 128, P, 0, None, None, 0, None) == 2
+    assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", P, 128, P, P, 17, 8, 128, P, 0, None, None, 0, None) == 2
     assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", P, 200, P, P, 4, 8, 200, P, 0, None, None, 0, None) == 2
     assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", P, 64, P, P, 4, 8, 128, P, 0, None, None, 0, None) == 2
     assert _st(lib, "i8q_gemm_w8a8_block_fused_quant", P, 128, P, P, 4, 8, 128, P, 0, None, P, 2, None) == 2
