@@ -414,13 +414,14 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_after();
         }
         for (int kb = 0; kb < KB; ++kb) {
+          // the stage first: it has normally landed long before, and a satisfied wait still costs
+          // this thread a few hundred cycles, which it then spends while the accumulator is busy
+          if (!mbar_wait(&full[stage], phase, SITE_FULL, abort_flag)) { ok = false; break; }
           if (BLOCKWISE) {
             // use u of buffer acc waits for the epilogue's u-th release (its bias initialisation)
             acc = acc_iter & 1;
             if (!mbar_wait(&tempty[acc], (acc_iter >> 1) & 1, SITE_TMEM_EMPTY, abort_flag)) { ok = false; break; }
-            tc_fence_after();
           }
-          if (!mbar_wait(&full[stage], phase, SITE_FULL, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);

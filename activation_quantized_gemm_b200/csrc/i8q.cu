@@ -629,20 +629,32 @@ i8q_status i8q_quant_weight_block(const uint16_t* w, int64_t N, int64_t K, int8_
   return I8Q_OK;
 }
 
+// stages (= warp pairs) per CTA of the FP8 block requantization: 12 x 16 KB per SM, 24 warps
+constexpr int REQUANT_NP = 12;
+
 i8q_status i8q_requant_fp8_to_int8_block(const uint8_t* w, const float* sf, int64_t N, int64_t K, int8_t* wq,
                                          float* sw, void* stream) {
   I8Q_REQUIRE(N >= 0 && K >= 0 && N < kMaxDim && K < kMaxDim && K % 128 == 0, I8Q_ERR_SHAPE);
+  I8Q_REQUIRE(cdiv(N, 128) * (K / 128) < kMaxDim, I8Q_ERR_SHAPE);   // block indices are 32-bit
   if (N == 0 || K == 0) return I8Q_OK;
   I8Q_REQUIRE(w && sf && wq && sw, I8Q_ERR_NULL);
   I8Q_REQUIRE(aligned16(w) && aligned16(sf) && aligned16(wq) && aligned16(sw), I8Q_ERR_ALIGN);
   int sms;
   i8q_status st = current_device(&sms);
   if (st) return st;
-  int64_t blocks = cdiv(N, 128) * (K / 128);
-  const int64_t cap = resident_grid(k_quant_weight_block<true>, 256, sms);
-  if (blocks > cap) blocks = cap;
-  k_quant_weight_block<true><<<(unsigned)blocks, 256, 0, S(stream)>>>(w, sf, (int)N, (int)K, wq, sw);
-  I8Q_LAUNCHED("k_quant_weight_block<e4m3>");
+  // one CTA per SM of REQUANT_NP warp pairs, each streaming its blocks through one TMA stage
+  using C = RequantCfg<REQUANT_NP>;
+  auto kern = k_requant_fp8_block<REQUANT_NP>;
+  const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
+  if (attr) return attr;
+  CUtensorMap tw;
+  st = make_tmap_2d(&tw, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, K, 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st) return st;
+  const int64_t nblocks = cdiv(N, 128) * (K / 128);
+  int64_t ctas = cdiv(nblocks, REQUANT_NP);
+  if (ctas > sms) ctas = sms;
+  kern<<<(unsigned)ctas, C::NUM_THREADS, C::SMEM_BYTES, S(stream)>>>(tw, sf, (int)N, (int)K, wq, sw);
+  I8Q_LAUNCHED("k_requant_fp8_block");
   return I8Q_OK;
 }
 

@@ -398,6 +398,174 @@ __global__ void __launch_bounds__(256) k_quant_weight_block(const void* __restri
 }
 
 // ----------------------------------------------------------------------------------------------
+// a3, TMA-fed: FP8-E4M3 -> BF16 -> INT8 128x128 block requantization, two warps per block.
+//
+// A CTA holds NP shared-memory stages of one 16 KB FP8 block each; a pair of warps owns a stage
+// and streams its blocks (gp, gp + TP, ... for global pair gp of TP) through it with TMA, warp h
+// of the pair taking rows 64 h .. 64 h + 63.  The two warps exchange their halves' code maxima
+// and, once both have finished with the block, the stage is refilled - two named barriers of 64
+// threads per block, no CTA-wide barrier.  Two warps per block keep the time a stage is occupied
+// by its quantization short, so that most of the NP stages of an SM are loading at any time.
+//
+// Block absmax from the codes: E4M3 -> f16 -> fp32 is exact and increasing in the code's magnitude
+// bits, and the fp32 product with |sf| and the bf16 rounding are monotone and odd, so the block's
+// max |bf16 value| is the dequantization of its largest code magnitude (NaN codes, 0x7F / 0xFF, are
+// outside the contract).  Pass 1 only takes byte maxima over the raw block.
+//
+// Codes by table: inside a block the INT8 code of an element is a function of its FP8 byte alone,
+// and odd in it (dequantization and quantization are both odd).  So each warp quantizes the 128
+// magnitudes once per block - with the same device arithmetic as the element-wise kernels, so the
+// table is bit-identical to what they compute per element - into a 128-byte table (one 32-bit
+// word per shared-memory bank: any lookup pattern is conflict-free).  Pass 2 then costs per
+// element one byte load from the table plus a few integer operations, instead of the
+// dequantization and the corrected quotient; the signs are applied to four packed codes at once.
+// A negative sf flips every sign: the table is built with |sf| and the sign bits are XORed.
+// Rows past N of the last block row arrive as zeros (TMA bounds fill) and are not written.
+// ----------------------------------------------------------------------------------------------
+template <int NP>
+struct RequantCfg {
+  static constexpr int BLOCK_BYTES = 128 * 128;
+  static constexpr int NUM_THREADS = 64 * NP;
+  static constexpr int TABLE_BYTES = 256;                  // per warp (128 used, 256-byte aligned)
+  static constexpr int XCH_BYTES = 8 * NP;                 // per pair: both warps' code maxima
+  static constexpr int BAR_BYTES = 8 * NP + 16;
+  static constexpr int SMEM_BYTES = NP * BLOCK_BYTES + 2 * NP * TABLE_BYTES + XCH_BYTES + BAR_BYTES + 1024;
+  static_assert(NP >= 1 && NP <= 15, "one named barrier per pair (ids 1 .. NP)");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+// largest E4M3 magnitude code (0..0x7E) among the 16 bytes of v, folded into two u16x2 maxima
+__device__ __forceinline__ void code_absmax16(const uint4& v, uint32_t& hi, uint32_t& lo) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t m = w[i] & 0x7F7F7F7Fu;
+    hi = max_u16x2(hi, m);                          // bytes 1 and 3 exact (bytes 0, 2 only break ties)
+    lo = max_u16x2(lo, __byte_perm(m, 0u, 0x2404)); // bytes 0 and 2 moved up, zeros below
+  }
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// Four codes of the FP8 word w from the magnitude table at shared address tbl (256-byte aligned):
+// table codes P (bytes 0..127), then negation of the bytes whose sign (w's, XOR sfm) is set and
+// whose code is not 0: -q = (q ^ 0xFF) + 1, carry-free for q >= 1.
+__device__ __forceinline__ uint32_t table_codes4(uint32_t w, uint32_t tbl, uint32_t sfm) {
+  const uint32_t wm = w & 0x7F7F7F7Fu;
+  const uint32_t c0 = lds_u8(prmt(wm, tbl, 0x7650u)), c1 = lds_u8(prmt(wm, tbl, 0x7651u));
+  const uint32_t c2 = lds_u8(prmt(wm, tbl, 0x7652u)), c3 = lds_u8(prmt(wm, tbl, 0x7653u));
+  const uint32_t P = prmt(prmt(c0, c1, 0x0040u), prmt(c2, c3, 0x0040u), 0x5410u);
+  const uint32_t nn = (P + 0x7F7F7F7Fu) & (w ^ sfm) & 0x80808080u;   // negative, non-zero code
+  const uint32_t mf = prmt(nn, 0u, 0xBA98u);                         // 0xFF in those bytes
+  return (P ^ mf) + (nn >> 7);
+}
+
+__device__ __forceinline__ void pair_sync(int id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); }
+
+template <int NP>
+__global__ void __launch_bounds__(RequantCfg<NP>::NUM_THREADS, 1)
+    k_requant_fp8_block(const __grid_constant__ CUtensorMap tmW, const float* __restrict__ sf, int N, int K,
+                        int8_t* __restrict__ wq, float* __restrict__ sw) {
+  using C = RequantCfg<NP>;
+  constexpr uint32_t kFailed = 0xFFFFFFFFu;                // exchange word of a warp whose wait expired
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tables = smem + NP * C::BLOCK_BYTES;
+  volatile uint32_t* xch = reinterpret_cast<volatile uint32_t*>(tables + 2 * NP * C::TABLE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(tables + 2 * NP * C::TABLE_BYTES + C::XCH_BYTES);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + NP);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int p = warp >> 1, h = warp & 1;
+  const int KB = K / 128;
+  const int nblocks = ((N + 127) / 128) * KB;
+  const int TP = gridDim.x * NP;
+  const int gp = blockIdx.x * NP + p;
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < NP; ++q) mbar_init(&full[q], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  uint64_t* bar = &full[p];
+  uint8_t* stage = smem + p * C::BLOCK_BYTES;
+  const uint8_t* half = stage + h * (C::BLOCK_BYTES / 2);
+  uint32_t* table = reinterpret_cast<uint32_t*>(tables + warp * C::TABLE_BYTES);
+  const uint32_t tbl = smem_u32(table);
+  volatile uint32_t* xs = xch + 2 * p;
+  const bool issuer = h == 0 && lane == 0;
+  const int nmine = gp < nblocks ? (nblocks - 1 - gp) / TP + 1 : 0;
+  auto issue = [&](int i) {                       // this pair's i-th block into its stage
+    const int b = gp + i * TP;
+    const int nb = b / KB, kb = b - nb * KB;
+    mbar_arrive_expect_tx(bar, C::BLOCK_BYTES);
+    tma_load_2d(stage, &tmW, bar, kb * 128, nb * 128);
+  };
+  if (issuer && nmine > 0) issue(0);
+  int i = 0;
+  for (; i < nmine; ++i) {
+    const int b = gp + i * TP;
+    const int nb = b / KB, kb = b - nb * KB;
+    const float scale = __ldg(sf + b);
+    const bool ok = warp_wait(bar, i & 1, SITE_FULL, abort_flag);
+    // pass 1: largest code magnitude of this warp's half
+    uint32_t m = 0;
+    if (ok) {
+      uint32_t hi = 0, lo = 0;
+#pragma unroll 8
+      for (int t = 0; t < 16; ++t) code_absmax16(*reinterpret_cast<const uint4*>(half + (t * 32 + lane) * 16), hi, lo);
+      m = max_u16x2(hi, lo);
+      m = max(m >> 24, (m >> 8) & 0xFFu);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) m = max(m, __shfl_xor_sync(FULL_MASK, m, off));
+    }
+    if (lane == 0) xs[h] = ok ? m : kFailed;
+    pair_sync(1 + p);
+    const uint32_t m0 = xs[0], m1 = xs[1];
+    if (m0 == kFailed || m1 == kFailed) break;    // both warps leave together
+    m = max(m0, m1);
+    const float asf = fabsf(scale);
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)m, __NV_E4M3);
+    const float cmax = __half2float(__low2half(*reinterpret_cast<const __half2*>(&hr)));
+    const QScale qs = make_qscale(__bfloat162float(__float2bfloat16_rn(__fmul_rn(cmax, asf))));
+    // the codes of magnitudes 4 lane .. 4 lane + 3 (element-wise arithmetic, |sf|)
+    {
+      uint32_t o[8];
+      e4m3x16_to_bf16x16(make_uint4(0x03020100u + 0x04040404u * (uint32_t)lane, 0u, 0u, 0u), asf, o);
+      table[lane] = quant_bf16x8(make_uint4(o[0], o[1], 0u, 0u), qs, true).x;
+    }
+    __syncwarp();
+    const uint32_t sfm = __float_as_uint(scale) >> 31 ? 0x80808080u : 0u;
+    // pass 2: 16 codes per lane per step; a warp step covers 4 rows of 128 bytes
+    const int row0 = nb * 128 + h * 64;
+    int8_t* dst0 = wq + (int64_t)row0 * K + kb * 128 + (lane & 7) * 16;
+#pragma unroll 4
+    for (int t = 0; t < 16; ++t) {
+      const int row = t * 4 + (lane >> 3);
+      const uint4 v = *reinterpret_cast<const uint4*>(half + (t * 32 + lane) * 16);
+      const uint4 c = make_uint4(table_codes4(v.x, tbl, sfm), table_codes4(v.y, tbl, sfm),
+                                 table_codes4(v.z, tbl, sfm), table_codes4(v.w, tbl, sfm));
+      if (row0 + row < N) *reinterpret_cast<uint4*>(dst0 + (int64_t)row * K) = c;
+    }
+    if (issuer) sw[b] = qs.s;
+    // both halves read (generic proxy) before TMA writes the stage again
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    pair_sync(1 + p);
+    if (issuer && i + 1 < nmine) issue(i + 1);
+  }
+  // a wait expired: the block in flight lands before the CTA exits
+  if (i < nmine && issuer) mbar_wait(bar, i & 1, SITE_DRAIN, nullptr);
+}
+
+// ----------------------------------------------------------------------------------------------
 // FP8 -> BF16 -> INT8 per-output-channel requantization: one CTA of 256 threads per weight row;
 // the second pass rebuilds the bf16 values from the FP8 bytes (re-read from L2).
 // ----------------------------------------------------------------------------------------------

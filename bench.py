@@ -60,7 +60,6 @@ def load_peaks():
 # bench's own command (profiles/<file>.md), keyed by (workload, M, N, K).  A kernel change
 # invalidates its entry: it must then be re-measured or removed (the line reports null).
 MEASURED_TRAFFIC = {
-    ("requant", 0, 18432, 7168): (217.65e6, "requant_fp8_block_n18432_k7168.md"),
     ("w8a16", 16, 12288, 4096): (51.30e6, "w8a16_m16_n12288_k4096.md"),
     ("w8a16", 16, 4096, 12288): (51.55e6, "w8a16_m16_n4096_k12288.md"),
 }

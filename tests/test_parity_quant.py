@@ -100,6 +100,27 @@ def test_requant_fp8_block(q, N, K):
     assert np.array_equal(host(sw), sw_ref)
 
 
+def test_requant_fp8_block_streams(q):
+    """More blocks than the kernel has warps (each warp streams several blocks through its stage),
+    a ragged last row-block, negative and zero block scales, an all-zero block and a block whose
+    largest magnitude is a subnormal code."""
+    N, K = 4100, 7168
+    w8, sf = synth.fp8_checkpoint(N, K, seed=41)
+    sf[1, 2] = -sf[1, 2]
+    sf[5, :] = -sf[5, :]
+    sf[3, 3] = 0.0
+    w8[256:384, 512:640] = 0
+    w8[0:128, 0:128] &= 0x87                      # E4M3 subnormals (exponent field 0) only
+    wq_ref, sw_ref = O.requant_fp8_to_int8_block(w8, sf)
+    wq = empty((N, K), torch.int8, 99)
+    sw = empty(sw_ref.shape, torch.float32)
+    q.i8q_requant_fp8_to_int8_block(dev(w8), dev(sf), wq, sw)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(sw).view(np.uint32), sw_ref.view(np.uint32))
+    bad = np.argwhere(host(wq) != wq_ref)
+    assert bad.size == 0, f"{len(bad)} codes differ, first at {bad[:4].tolist()}"
+
+
 def test_requant_fp8_all_codes(q):
     """Every finite E4M3 code appears, including subnormals and +-448."""
     codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
