@@ -130,22 +130,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
 }
 
 // 4 signed int8 (one 32-bit word) -> 4 exact bf16 values as two bf16x2 words.  bf16 has 8
-// significant bits, so |q| <= 127 is exact but the f16 offset trick below does not fit: the
-// magnitude m = |q| (per byte: x ^ mask + (mask & 1), no carry between bytes) goes into the
-// mantissa of 128.0 (bf16 0x4300 | m = 128 + m, m < 128), 128 is subtracted (exact), and the sign
-// bit of q is put back.
+// significant bits, so |q| <= 127 is exact, but the offset-binary trick of the f16 version below
+// does not fit in its 7-bit mantissa (q + 128 spans two binades).
 __device__ __forceinline__ void i8x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const uint32_t sg = w & 0x80808080u;
-  const uint32_t t = sg >> 7;                       // 1 in each negative byte
-  const uint32_t mag = (w ^ (t * 0xFFu)) + t;       // per-byte |q|
-  const uint32_t a = __byte_perm(mag, 0x43434343u, 0x4140);
-  const uint32_t b = __byte_perm(mag, 0x43434343u, 0x4342);
-  const __nv_bfloat162 c128 = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)0x4300),
-                                                 __ushort_as_bfloat16((unsigned short)0x4300));
-  __nv_bfloat162 ha = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&a), c128);
-  __nv_bfloat162 hb = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&b), c128);
-  lo = *reinterpret_cast<uint32_t*>(&ha) | __byte_perm(sg, 0u, 0x1404);
-  hi = *reinterpret_cast<uint32_t*>(&hb) | __byte_perm(sg, 0u, 0x3424);
+  // a code q with sign bit s and low bits l is l - 128 s.  With 0x43 as the high byte, bf16
+  // 0x43 | l is 128 + l and 0x43 | (s << 7) is 128 or 256 (all exact), so one packed subtract of
+  // the two gives q exactly (+0 for q = 0).
+  const uint32_t pl = __byte_perm(w, 0x43434343u, 0x4140), ph = __byte_perm(w, 0x43434343u, 0x4342);
+  const uint32_t al = pl & 0xFF7FFF7Fu, sl = pl & 0xFF80FF80u, ah = ph & 0xFF7FFF7Fu, sh = ph & 0xFF80FF80u;
+  __nv_bfloat162 ha = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&al), *reinterpret_cast<const __nv_bfloat162*>(&sl));
+  __nv_bfloat162 hb = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&ah), *reinterpret_cast<const __nv_bfloat162*>(&sh));
+  lo = *reinterpret_cast<uint32_t*>(&ha);
+  hi = *reinterpret_cast<uint32_t*>(&hb);
 }
 
 // Group scale (fp16 or bf16 bits) -> fp32 (exact), and fp32 -> output bits (round to nearest even).

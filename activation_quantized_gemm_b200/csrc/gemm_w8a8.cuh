@@ -25,8 +25,8 @@
 //                accumulator buffer by arriving on the leader's barrier.
 // Register split: warpgroup 0 drops to 56 registers per thread, the epilogue warpgroups rise to
 // 224 (block-wise keeps a 128-column fp32 running sum per thread).
-// Tiles are visited in bands of 8 pair-rows (2048 tokens) so that the activations and weights in
-// use by all pairs at one time stay resident in L2.
+// Tiles are visited in bands of 16 pair-rows (4096 tokens): the band's activations stay resident
+// in L2 while the weights stream through it once per band.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -37,7 +37,7 @@ namespace i8q {
 
 constexpr int GEMM_BM = 256;       // tokens per pair tile (MMA M, cta_group::2)
 constexpr int GEMM_BK = 128;       // K per slab (bytes of int8 = one 128B swizzle row)
-constexpr int GEMM_GROUP_M = 8;    // pair-tile rows per raster band
+constexpr int GEMM_GROUP_M = 16;   // pair-tile rows per raster band
 constexpr int kMaxExperts = 1024;  // grouped (MoE) GEMMs: experts per call
 
 template <int BN>

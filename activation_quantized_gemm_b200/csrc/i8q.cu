@@ -215,6 +215,23 @@ static i8q_status launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned blo
   I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
   return I8Q_OK;
 }
+// The same with dynamic shared memory.
+template <typename... KArgs, typename... Args>
+static i8q_status launch_pdl_smem(void (*kern)(KArgs...), unsigned grid, unsigned block, int smem, cudaStream_t s,
+                                  Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
+  return I8Q_OK;
+}
 
 // ------------------------------------------------------------------ W8A16 launch ------------
 // Split-K factor of the W8A16 GEMM: the largest cluster size s in 1..8 (and <= K / 128) whose
@@ -653,7 +670,8 @@ i8q_status i8q_requant_fp8_to_int8_block(const uint8_t* w, const float* sf, int6
   const int64_t nblocks = cdiv(N, 128) * (K / 128);
   int64_t ctas = cdiv(nblocks, REQUANT_NP);
   if (ctas > sms) ctas = sms;
-  kern<<<(unsigned)ctas, C::NUM_THREADS, C::SMEM_BYTES, S(stream)>>>(tw, sf, (int)N, (int)K, wq, sw);
+  st = launch_pdl_smem(kern, (unsigned)ctas, C::NUM_THREADS, C::SMEM_BYTES, S(stream), tw, sf, (int)N, (int)K, wq, sw);
+  if (st) return st;
   I8Q_LAUNCHED("k_requant_fp8_block");
   return I8Q_OK;
 }

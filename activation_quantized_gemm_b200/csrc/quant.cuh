@@ -489,12 +489,16 @@ __global__ void __launch_bounds__(RequantCfg<NP>::NUM_THREADS, 1)
   const int nblocks = ((N + 127) / 128) * KB;
   const int TP = gridDim.x * NP;
   const int gp = blockIdx.x * NP + p;
+  // Launched with programmatic stream serialization: the set-up below overlaps the end of the
+  // kernel before it, and no global memory is touched before that kernel has completed.
+  grid_dependents_launch();
   if (threadIdx.x == 0) {
     for (int q = 0; q < NP; ++q) mbar_init(&full[q], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
+  grid_dependency_wait();
   uint64_t* bar = &full[p];
   uint8_t* stage = smem + p * C::BLOCK_BYTES;
   const uint8_t* half = stage + h * (C::BLOCK_BYTES / 2);
