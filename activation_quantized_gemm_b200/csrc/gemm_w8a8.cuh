@@ -40,22 +40,30 @@ constexpr int GEMM_BK = 128;       // K per slab (bytes of int8 = one 128B swizz
 constexpr int GEMM_GROUP_M = 16;   // pair-tile rows per raster band
 constexpr int kMaxExperts = 1024;  // grouped (MoE) GEMMs: experts per call
 
-template <int BN>
+// TS (block-wise bf16 output): the epilogue hands each finished tile to TMA stores from a 64 KB
+// output buffer instead of storing it itself, so that the MMAs of the next tile do not wait for
+// the tile-end write burst (every SM finishes its tile at about the same time); one stage of the
+// ring gives way for the buffer.
+template <int BN, bool TS = false>
 struct W8A8Cfg {
   static constexpr int A_BYTES = 128 * GEMM_BK;          // this CTA's 128 token rows
   static constexpr int B_BYTES = (BN / 2) * GEMM_BK;     // this CTA's BN/2 weight rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = 6;
+  static constexpr int STAGES = TS ? 5 : 6;
   static constexpr int TMEM_COLS = 512;                  // two accumulator buffers of BN columns
   static constexpr int NUM_THREADS = 384;
   static constexpr int EPI_WARPS = 8;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int EPI_STAGE_BYTES = EPI_WARPS * 32 * 80;   // per epilogue warp: 32 rows x 80 B
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + EPI_STAGE_BYTES + 1024;  // + alignment slack
+  static constexpr int OUT_WARP_BYTES = 32 * (BN / 2) * 2;          // TS: a warp's 32 rows x BN/2 bf16
+  static constexpr int OUT_BYTES = TS ? EPI_WARPS * OUT_WARP_BYTES : 0;
+  static constexpr int EPI_STAGE_BYTES = TS ? 0 : EPI_WARPS * 32 * 80;   // per epilogue warp: 32 rows x 80 B
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BYTES + BAR_BYTES + EPI_STAGE_BYTES + 1024;  // + alignment slack
   // grouped (MoE) problems: per-expert row offsets and m-tile prefix sums, kMaxExperts + 1 each
   static constexpr int GROUP_BYTES = 2 * (kMaxExperts + 1) * 4;
   static constexpr int SMEM_BYTES_GROUPED = SMEM_BYTES + GROUP_BYTES;
   static_assert(2 * BN <= TMEM_COLS, "two accumulators must fit in TMEM");
+  static_assert(!TS || BN == 256, "TMA-store epilogue: two 64-column boxes per warp");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(BN % 32 == 0 && BN <= 256, "MMA N (each CTA's BN / 2 weight rows: whole 8-row groups)");
 };
 
@@ -143,6 +151,18 @@ __device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t v) {
       "r"(v)
       : "memory");
 }
+
+// TMA tile store shared -> global (bulk async-group of the issuing thread; parts of the box
+// outside the tensor are not written), and the waits on this thread's groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_inc() {
@@ -296,22 +316,24 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 template <int BN, bool BLOCKWISE, bool OUT_F32, bool DEBUG, bool GROUPED = false, bool ALIGNED = true>
 __global__ void __launch_bounds__(384, 1)
     k_gemm_w8a8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const W8A8Args args) {
-  using C = W8A8Cfg<BN>;
+                const __grid_constant__ CUtensorMap tmY, const W8A8Args args) {
+  constexpr bool TS = BLOCKWISE && !OUT_F32 && !GROUPED && ALIGNED;   // TMA-store epilogue (tmY)
+  using C = W8A8Cfg<BN, TS>;
   static_assert(!BLOCKWISE || BN == 256, "block-wise pair tiles are two weight blocks wide");
   constexpr int HALF = BN / 2;                 // columns per epilogue warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* sOut = smem + C::STAGES * C::STAGE_BYTES;   // TS: output boxes (1024-byte aligned)
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::OUT_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* done = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint8_t* sStage = smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES;
+  uint8_t* sStage = smem + C::STAGES * C::STAGE_BYTES + C::OUT_BYTES + C::BAR_BYTES;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cta_rank_in_cluster();
@@ -621,6 +643,29 @@ __global__ void __launch_bounds__(384, 1)
               }
             }
           }
+        } else if constexpr (TS) {
+          // the warp's 32 rows x 128 columns as two 128B-swizzled boxes of 32 x 64 bf16 (row = lane:
+          // 16-byte chunk c of a row at chunk c ^ (row % 8)), then two TMA stores.  The buffer is
+          // rewritten only once the previous tile's stores have read it.
+          uint8_t* obuf = sOut + (warp - 4) * C::OUT_WARP_BYTES;
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 2; ++k)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int j = 32 * k + 4 * c;
+              *reinterpret_cast<uint4*>(obuf + k * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(pack_bf16x2(sum[j].x, sum[j].y), pack_bf16x2(sum[j + 1].x, sum[j + 1].y),
+                             pack_bf16x2(sum[j + 2].x, sum[j + 2].y), pack_bf16x2(sum[j + 3].x, sum[j + 3].y));
+            }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0 && m - lane < row_end) {
+            if (n0 < N) tma_store_2d(&tmY, obuf, n0, m - lane);
+            if (n0 + 64 < N) tma_store_2d(&tmY, obuf + 4096, n0 + 64, m - lane);
+            bulk_commit();
+          }
         } else {
 #pragma unroll
           for (int c = 0; c < HALF / 32; ++c) {
@@ -632,6 +677,11 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
+    }
+    // the last tiles' stores complete (and stop reading shared memory) before the CTA can exit
+    if constexpr (TS) {
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
     }
   }
 

@@ -319,17 +319,25 @@ static i8q_status gemm_w8a8_common_checks(const int8_t* xq, const float* sx, con
 
 template <int BN, bool BLOCKWISE, bool F32, bool DBG, bool ALIGNED = true>
 static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms, cudaStream_t s) {
-  using C = W8A8Cfg<BN>;
+  constexpr bool TS = BLOCKWISE && !F32 && ALIGNED;   // the kernel's TMA-store epilogue (non-grouped)
+  using C = W8A8Cfg<BN, TS>;
   auto kern = k_gemm_w8a8<BN, BLOCKWISE, F32, DBG, false, ALIGNED>;
   const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
   if (attr) return attr;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
   i8q_status st = make_tmap_2d(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, a.K, 128, GEMM_BK,
                                CU_TENSOR_MAP_SWIZZLE_128B);
   if (st) return st;
   st = make_tmap_2d(&tb, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.N, a.K, a.K, BN / 2, GEMM_BK,
                     CU_TENSOR_MAP_SWIZZLE_128B);
   if (st) return st;
+  if constexpr (TS) {
+    // bf16 output tiles of 32 rows x 64 columns (128 bytes: the 128-byte swizzle span); N % 8 == 0
+    st = make_tmap_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.N, a.N, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st) return st;
+  } else {
+    ty = ta;   // unused
+  }
   const int64_t tiles = cdiv(a.M, GEMM_BM) * cdiv(a.N, BN);
   const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
   cudaLaunchConfig_t cfg = {};
@@ -346,7 +354,7 @@ static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, a));
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, a));
   return I8Q_OK;
 }
 
@@ -385,7 +393,7 @@ static i8q_status launch_w8a8_grouped(const int8_t* xq, const int8_t* wq, const 
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, a));
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, ta, a));   // no TMA-store epilogue: tmY unused
   return I8Q_OK;
 }
 
