@@ -22,9 +22,10 @@
 //                accumulator-ready signals to both CTAs.
 //   warps 4..11  epilogue: warp w reads TMEM lane quarter (w % 4) (tile rows) and column half
 //                (w - 4) / 4; one row per thread.  Both CTAs' epilogue warps release an
-//                accumulator buffer by arriving on the leader's barrier.
-// Register split: warpgroup 0 drops to 56 registers per thread, the epilogue warpgroups rise to
-// 224 (block-wise keeps a 128-column fp32 running sum per thread).
+//                accumulator buffer by arriving on the leader's barrier.  Block-wise bf16 tiles
+//                leave through TMA stores from per-warp shared-memory boxes (see W8A8Cfg).
+// Register split: warpgroup 0 drops to 24 registers per thread, the epilogue warpgroups rise to
+// 240 (block-wise keeps a 128-column fp32 running sum per thread).
 // Tiles are visited in bands of 16 pair-rows (4096 tokens): the band's activations stay resident
 // in L2 while the weights stream through it once per band.
 #pragma once

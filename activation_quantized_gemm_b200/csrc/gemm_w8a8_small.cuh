@@ -13,7 +13,8 @@
 //               sx[m] * sw[n].  Block-wise: each 128-K slab has its own TMEM accumulator; its int32
 //               partial sums are folded into fp32 running sums with sx[m][kb] * sw[n/128][kb].
 //   next warp   TMA producer: weight slab [128 rows x 128 K] + activation slab [MP x 128 K].
-//   last warp   TMEM allocation and MMA issue (4 x tcgen05.mma per slab).
+//   next warp   TMEM allocation and MMA issue (4 x tcgen05.mma per slab).
+//   (FUSEDQ)    four quantizer warps after those.
 // Two CTAs share an SM for up to 64 tokens (rings of 4..6 stages each), one CTA for 128 (TMEM and
 // registers); the launch keeps all CTAs in one wave.
 //
