@@ -21,7 +21,9 @@
 // pattern is that integer's two's-complement int8 code.
 //
 // Memory side: 16-byte vector loads, several in flight per thread (the next row / block is
-// loaded while the current one is quantized), codes written as 8- or 16-byte vectors.
+// loaded while the current one is quantized), codes written as 8- or 16-byte vectors.  The FP8
+// block requantization instead streams whole 128x128 blocks into shared memory with TMA and turns
+// each block into a code table (k_requant_fp8_block below).
 #pragma once
 
 #include <cuda_bf16.h>
