@@ -159,7 +159,7 @@ def i8q_gemm_w8a8_block(xq, sx, wq, sw, y, out: int = I8Q_OUT_BF16, debug_partia
 
 def i8q_gemm_w8a8_block_fused_quant(x, wq, sw, y, out: int = I8Q_OUT_BF16, xq_out=None, sx_out=None,
                                     ld_sx: Optional[int] = None, stream=None) -> None:
-    """y [M, N] = block-wise W8A8 GEMM of bf16 x [M, K] (M <= 64) with the per-token-group
+    """y [M, N] = block-wise W8A8 GEMM of bf16 x [M, K] (1 <= M <= 16) with the per-token-group
     quantization done inside the GEMM; xq_out [M, K] / sx_out [K/128, ld_sx] optionally receive the
     quantized activations."""
     M, K = x.shape
