@@ -647,10 +647,10 @@ i8q_status i8q_quant_weight_block(const uint16_t* w, int64_t N, int64_t K, int8_
   i8q_status st = current_device(&sms);
   if (st) return st;
   int64_t blocks = cdiv(N, 128) * (K / 128);
-  const int64_t cap = resident_grid(k_quant_weight_block<false>, 256, sms);
+  const int64_t cap = resident_grid(k_quant_weight_block, 256, sms);
   if (blocks > cap) blocks = cap;
-  k_quant_weight_block<false><<<(unsigned)blocks, 256, 0, S(stream)>>>(w, nullptr, (int)N, (int)K, wq, sw);
-  I8Q_LAUNCHED("k_quant_weight_block<bf16>");
+  k_quant_weight_block<<<(unsigned)blocks, 256, 0, S(stream)>>>(w, (int)N, (int)K, wq, sw);
+  I8Q_LAUNCHED("k_quant_weight_block");
   return I8Q_OK;
 }
 

@@ -319,83 +319,49 @@ __device__ __forceinline__ void e4m3x16_to_bf16x16(const uint4& v, float scale, 
 }
 
 // ----------------------------------------------------------------------------------------------
-// a3 / a3': 128x128 block quantization, one CTA of 256 threads per block, persistent over blocks
-// (the next block's input is loaded while the current one is quantized).
-// FP8 == true : E4M3 bytes with fp32 block scales sf, dequantized to bf16 first.
-// FP8 == false: bf16 input.
-// Each thread owns 64 values of the block as 8 bf16x8 vectors; rows past N (partial last block)
-// are neither read nor written.
+// a3': 128x128 block quantization of a bf16 weight, one CTA of 256 threads per block, persistent
+// over blocks (the next block's input is loaded while the current one is quantized).  Thread t
+// owns 64 values of the block as 8 bf16x8 vectors (vector j: row (t + 256 j) / 16, elements
+// (t % 16) * 8 .. +8); rows past N (partial last block) are neither read nor written.
 // ----------------------------------------------------------------------------------------------
-template <bool FP8>
-__global__ void __launch_bounds__(256) k_quant_weight_block(const void* __restrict__ w, const float* __restrict__ sf,
-                                                            int N, int K, int8_t* __restrict__ wq,
-                                                            float* __restrict__ sw) {
-  constexpr int RAW = FP8 ? 4 : 8;            // 16-byte input vectors per thread per block
+__global__ void __launch_bounds__(256) k_quant_weight_block(const uint16_t* __restrict__ w, int N, int K,
+                                                            int8_t* __restrict__ wq, float* __restrict__ sw) {
   __shared__ float red[8];
   const int KB = K / 128;
   const int nblocks = ((N + 127) / 128) * KB;
-  // fp8: vector j of thread t covers row (t + 256 j) / 8, bytes (t % 8) * 16 .. +16
-  // bf16: vector j covers row (t + 256 j) / 16, elements (t % 16) * 8 .. +8
-  auto row_of = [&](int j) { return FP8 ? (int)((threadIdx.x + 256 * j) >> 3) : (int)((threadIdx.x + 256 * j) >> 4); };
-  auto col_of = [&](int j) { return FP8 ? (int)((threadIdx.x & 7) * 16) : (int)((threadIdx.x & 15) * 8); };
-  auto load = [&](int b, uint4 (&raw)[RAW]) {
+  auto row_of = [&](int j) { return (int)((threadIdx.x + 256 * j) >> 4); };
+  const int col = (int)((threadIdx.x & 15) * 8);
+  auto load = [&](int b, uint4 (&raw)[8]) {
     const int nb = b / KB, kb = b - (b / KB) * KB;
 #pragma unroll
-    for (int j = 0; j < RAW; ++j) {
+    for (int j = 0; j < 8; ++j) {
       const int row = nb * 128 + row_of(j);
       raw[j] = make_uint4(0, 0, 0, 0);
-      if (b < nblocks && row < N) {
-        if constexpr (FP8)
-          raw[j] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(w) + (int64_t)row * K +
-                                                        kb * 128 + col_of(j)));
-        else
-          raw[j] = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(w) + (int64_t)row * K +
-                                                        kb * 128 + col_of(j)));
-      }
+      if (b < nblocks && row < N) raw[j] = __ldg(reinterpret_cast<const uint4*>(w + (int64_t)row * K + kb * 128 + col));
     }
   };
-  uint4 cur[RAW], nxt[RAW];
+  uint4 cur[8], nxt[8];
   int b = blockIdx.x;
   load(b, cur);
   for (; b < nblocks; b += gridDim.x) {
     load(b + gridDim.x, nxt);
     const int nb = b / KB, kb = b - (b / KB) * KB;
-    uint4 v[8];                                 // 64 bf16 values
-    if constexpr (FP8) {
-      const float scale = __ldg(sf + b);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t o[8];
-        e4m3x16_to_bf16x16(cur[j], scale, o);
-        v[2 * j] = make_uint4(o[0], o[1], o[2], o[3]);
-        v[2 * j + 1] = make_uint4(o[4], o[5], o[6], o[7]);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = cur[j];
-    }
     float a = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) a = fmaxf(a, absmax_bf16x8(v[j]));
+    for (int j = 0; j < 8; ++j) a = fmaxf(a, absmax_bf16x8(cur[j]));
     a = block_absmax(a, red, 8);
     const QScale qs = make_qscale(a);
 #pragma unroll
-    for (int j = 0; j < RAW; ++j) {
+    for (int j = 0; j < 8; ++j) {
       const int row = nb * 128 + row_of(j);
       const bool ok = row < N;
-      int8_t* dst = wq + (int64_t)row * K + kb * 128 + col_of(j);
-      if constexpr (FP8) {
-        const uint2 lo = quant_bf16x8(v[2 * j], qs, ok), hi = quant_bf16x8(v[2 * j + 1], qs, ok);
-        if (ok) *reinterpret_cast<uint4*>(dst) = make_uint4(lo.x, lo.y, hi.x, hi.y);
-      } else {
-        const uint2 c = quant_bf16x8(v[j], qs, ok);
-        if (ok) *reinterpret_cast<uint2*>(dst) = c;
-      }
+      const uint2 c = quant_bf16x8(cur[j], qs, ok);
+      if (ok) *reinterpret_cast<uint2*>(wq + (int64_t)row * K + kb * 128 + col) = c;
     }
     if (threadIdx.x == 0) sw[b] = qs.s;
     __syncthreads();                            // red[] is reused by the next block
 #pragma unroll
-    for (int j = 0; j < RAW; ++j) cur[j] = nxt[j];
+    for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
   }
 }
 
