@@ -106,6 +106,35 @@ def test_fp8_block_absmax_is_the_largest_code_dequantized():
             assert float(mag[blk].max()) == expect
 
 
+def test_requant_codes_are_an_odd_function_of_the_byte():
+    """Within a 128x128 block the requantized code of an element depends on its E4M3 byte alone and
+    is odd in it: q(b | 0x80) = -q(b & 0x7F).  Dequantization (an fp32 product and a bf16 rounding)
+    and quantization (an IEEE quotient, half-to-even, clamp) are both odd, and the block scale is
+    shared, so a per-block table of 128 magnitude codes reproduces every element.  Checked on
+    blocks with positive, negative and zero scales, every finite code in each block, and on the
+    block absmax taken from the largest code magnitude with |sf|."""
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    w8 = np.resize(codes, (256, 512)).astype(np.uint8)
+    rng = np.random.default_rng(23)
+    rng.shuffle(w8.reshape(-1))
+    sf = np.array([[0.5, -3.0e-3, 0.0, -7.5], [2.0 ** -20, -0.25, 1.0e-2, 3.0]], np.float32)
+    wq, sw = O.requant_fp8_to_int8_block(w8, sf)
+    for i in range(2):
+        for j in range(4):
+            blk = (slice(i * 128, (i + 1) * 128), slice(j * 128, (j + 1) * 128))
+            b, q = w8[blk].ravel(), wq[blk].ravel().astype(int)
+            table = {}
+            for bb, qq in zip(b.tolist(), q.tolist()):
+                assert table.setdefault(bb, qq) == qq, (i, j, bb)
+            for bb, qq in table.items():
+                if bb & 0x80 and (bb & 0x7F) in table:
+                    assert qq == -table[bb & 0x7F], (i, j, bb)
+            # the block scale from the largest magnitude code and |sf|
+            top = np.array([[int((b & 0x7F).max())]], np.uint8)
+            a = float(O.bf16_to_f32(O.dequant_fp8_block_to_bf16(top, np.abs(sf[i:i + 1, j:j + 1])))[0, 0])
+            assert sw[i, j] == np.float32(a) / np.float32(127.0), (i, j)
+
+
 def test_requant_is_dequant_then_block_quant():
     w8, sf = synth.fp8_checkpoint(256, 256, seed=15)
     wq, sw = O.requant_fp8_to_int8_block(w8, sf)
