@@ -41,30 +41,33 @@ constexpr int GEMM_BK = 128;       // K per slab (bytes of int8 = one 128B swizz
 constexpr int GEMM_GROUP_M = 16;   // pair-tile rows per raster band
 constexpr int kMaxExperts = 1024;  // grouped (MoE) GEMMs: experts per call
 
-// TS (block-wise bf16 output): the epilogue hands each finished tile to TMA stores from a 64 KB
-// output buffer instead of storing it itself, so that the MMAs of the next tile do not wait for
-// the tile-end write burst (every SM finishes its tile at about the same time); one stage of the
-// ring gives way for the buffer.
-template <int BN, bool TS = false>
+// OUT_MODE 1 and 2 (block-wise bf16 output): the epilogue hands each finished tile to TMA stores
+// from a 64 KB output buffer instead of storing it itself, so that the MMAs of the next tile do not
+// wait for the tile-end write burst (every SM finishes its tile at about the same time).  1 (dense):
+// one stage of the ring gives way for the buffer.  2 (grouped): a store box must not cross into the
+// next expert's rows, so warps whose 32 rows straddle an expert boundary keep the direct stores
+// (and their staging slab); two stages give way.  0: direct stores.
+template <int BN, int OUT_MODE = 0>
 struct W8A8Cfg {
   static constexpr int A_BYTES = 128 * GEMM_BK;          // this CTA's 128 token rows
   static constexpr int B_BYTES = (BN / 2) * GEMM_BK;     // this CTA's BN/2 weight rows
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = TS ? 5 : 6;
+  static constexpr bool TS = OUT_MODE != 0;
+  static constexpr int STAGES = OUT_MODE == 0 ? 6 : (OUT_MODE == 1 ? 5 : 4);
   static constexpr int TMEM_COLS = 512;                  // two accumulator buffers of BN columns
   static constexpr int NUM_THREADS = 384;
   static constexpr int EPI_WARPS = 8;
   static constexpr int BAR_BYTES = 256;
   static constexpr int OUT_WARP_BYTES = 32 * (BN / 2) * 2;          // TS: a warp's 32 rows x BN/2 bf16
   static constexpr int OUT_BYTES = TS ? EPI_WARPS * OUT_WARP_BYTES : 0;
-  static constexpr int EPI_STAGE_BYTES = TS ? 0 : EPI_WARPS * 32 * 80;   // per epilogue warp: 32 rows x 80 B
+  static constexpr int EPI_STAGE_BYTES = OUT_MODE == 1 ? 0 : EPI_WARPS * 32 * 80;   // per epilogue warp: 32 rows x 80 B
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + OUT_BYTES + BAR_BYTES + EPI_STAGE_BYTES + 1024;  // + alignment slack
   // grouped (MoE) problems: per-expert row offsets and m-tile prefix sums, kMaxExperts + 1 each
   static constexpr int GROUP_BYTES = 2 * (kMaxExperts + 1) * 4;
   static constexpr int SMEM_BYTES_GROUPED = SMEM_BYTES + GROUP_BYTES;
   static_assert(2 * BN <= TMEM_COLS, "two accumulators must fit in TMEM");
   static_assert(!TS || BN == 256, "TMA-store epilogue: two 64-column boxes per warp");
-  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert((OUT_MODE == 1 ? SMEM_BYTES : SMEM_BYTES_GROUPED) <= 232448, "shared memory");
   static_assert(BN % 32 == 0 && BN <= 256, "MMA N (each CTA's BN / 2 weight rows: whole 8-row groups)");
 };
 
@@ -318,8 +321,8 @@ template <int BN, bool BLOCKWISE, bool OUT_F32, bool DEBUG, bool GROUPED = false
 __global__ void __launch_bounds__(384, 1)
     k_gemm_w8a8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmY, const W8A8Args args) {
-  constexpr bool TS = BLOCKWISE && !OUT_F32 && !GROUPED && ALIGNED;   // TMA-store epilogue (tmY)
-  using C = W8A8Cfg<BN, TS>;
+  constexpr bool TS = BLOCKWISE && !OUT_F32 && ALIGNED;   // TMA-store epilogue (tmY)
+  using C = W8A8Cfg<BN, TS ? (GROUPED ? 2 : 1) : 0>;
   static_assert(!BLOCKWISE || BN == 256, "block-wise pair tiles are two weight blocks wide");
   constexpr int HALF = BN / 2;                 // columns per epilogue warp
   extern __shared__ uint8_t smem_raw[];
@@ -644,10 +647,11 @@ __global__ void __launch_bounds__(384, 1)
               }
             }
           }
-        } else if constexpr (TS) {
+        } else if (TS && (!GROUPED || m - lane + 32 <= row_end || row_end >= M)) {
           // the warp's 32 rows x 128 columns as two 128B-swizzled boxes of 32 x 64 bf16 (row = lane:
-          // 16-byte chunk c of a row at chunk c ^ (row % 8)), then two TMA stores.  The buffer is
-          // rewritten only once the previous tile's stores have read it.
+          // 16-byte chunk c of a row at chunk c ^ (row % 8)), then two TMA stores (rows >= M and
+          // columns >= N are clipped by the tensor map; grouped: only boxes inside the expert's rows).
+          // The buffer is rewritten only once the previous tile's stores have read it.
           uint8_t* obuf = sOut + (warp - 4) * C::OUT_WARP_BYTES;
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();

@@ -319,8 +319,8 @@ static i8q_status gemm_w8a8_common_checks(const int8_t* xq, const float* sx, con
 
 template <int BN, bool BLOCKWISE, bool F32, bool DBG, bool ALIGNED = true>
 static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms, cudaStream_t s) {
-  constexpr bool TS = BLOCKWISE && !F32 && ALIGNED;   // the kernel's TMA-store epilogue (non-grouped)
-  using C = W8A8Cfg<BN, TS>;
+  constexpr bool TS = BLOCKWISE && !F32 && ALIGNED;   // the kernel's TMA-store epilogue
+  using C = W8A8Cfg<BN, TS ? 1 : 0>;
   auto kern = k_gemm_w8a8<BN, BLOCKWISE, F32, DBG, false, ALIGNED>;
   const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES);
   if (attr) return attr;
@@ -361,22 +361,28 @@ static i8q_status launch_w8a8(const int8_t* xq, const int8_t* wq, const W8A8Args
 // Grouped (MoE) problems: the pair-tile kernel with the expert map.  The number of m-tiles is
 // known only on the device (the offsets are device data), so the grid covers the worst case:
 // every expert may add one partial m-tile, ceil(M / 256) + E m-tiles in all.
-template <bool BLOCKWISE, bool F32, bool DBG>
-static i8q_status launch_w8a8_grouped(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms,
-                                      cudaStream_t s) {
+template <bool BLOCKWISE, bool F32, bool DBG, bool ALIGNED>
+static i8q_status launch_w8a8_grouped_k(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms,
+                                        cudaStream_t s) {
   constexpr int BN = 256;
-  using C = W8A8Cfg<BN>;
-  auto kern = a.N % 8 == 0 ? k_gemm_w8a8<BN, BLOCKWISE, F32, DBG, true, true>
-                           : k_gemm_w8a8<BN, BLOCKWISE, F32, DBG, true, false>;
+  constexpr bool TS = BLOCKWISE && !F32 && ALIGNED;   // the kernel's TMA-store epilogue
+  using C = W8A8Cfg<BN, TS ? 2 : 0>;
+  auto kern = k_gemm_w8a8<BN, BLOCKWISE, F32, DBG, true, ALIGNED>;
   const i8q_status attr = ensure_smem(kern, C::SMEM_BYTES_GROUPED);
   if (attr) return attr;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
   i8q_status st = make_tmap_2d(&ta, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.M, a.K, a.K, 128, GEMM_BK,
                                CU_TENSOR_MAP_SWIZZLE_128B);
   if (st) return st;
   st = make_tmap_2d(&tb, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.E * a.N, a.K, a.K, BN / 2, GEMM_BK,
                     CU_TENSOR_MAP_SWIZZLE_128B);
   if (st) return st;
+  if constexpr (TS) {
+    st = make_tmap_2d(&ty, a.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.M, a.N, a.N, 32, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st) return st;
+  } else {
+    ty = ta;   // unused
+  }
   const int64_t tiles = (cdiv(a.M, GEMM_BM) + a.E) * cdiv(a.N, BN);
   const int64_t pairs = tiles < sms / 2 ? tiles : sms / 2;
   cudaLaunchConfig_t cfg = {};
@@ -393,8 +399,15 @@ static i8q_status launch_w8a8_grouped(const int8_t* xq, const int8_t* wq, const 
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, ta, a));   // no TMA-store epilogue: tmY unused
+  I8Q_CUDA(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, a));
   return I8Q_OK;
+}
+
+template <bool BLOCKWISE, bool F32, bool DBG>
+static i8q_status launch_w8a8_grouped(const int8_t* xq, const int8_t* wq, const W8A8Args& a, int sms,
+                                      cudaStream_t s) {
+  if (a.N % 8 == 0) return launch_w8a8_grouped_k<BLOCKWISE, F32, DBG, true>(xq, wq, a, sms, s);
+  return launch_w8a8_grouped_k<BLOCKWISE, F32, DBG, false>(xq, wq, a, sms, s);
 }
 
 static i8q_status grouped_checks(const int32_t* off, int64_t E, int64_t M, int64_t N, int64_t K) {
